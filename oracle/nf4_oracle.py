@@ -1,0 +1,390 @@
+"""Plain CPU oracle for the QLoRA NF4 frozen-base linear layer.
+
+TEST INFRASTRUCTURE ONLY. This module is the slow, obviously correct reference that
+the CUDA library is checked against. Only the test suite, the smoke check in
+``__graft_entry__`` and the CPU-baseline leg of ``bench.py`` may import it. The product
+path (the C-ABI library and its Python binding) never imports, calls or links it, and it
+shares no code, table or constant generator with that path.
+
+Precision: encodings (codebook, codes, 8-bit scales, dequantized bf16) are computed in the
+fp32 arithmetic the method fixes, with every fp32 operation written out; products are
+computed in fp64 from the exact inputs.
+
+Sources (web pages on QLoRA, Dettmers et al., arXiv:2305.14314), cited by page title and
+section:
+
+* "QLoRA in LLMs" (tensortonic.com): §2 "How Quantization Works" (absmax scale, round,
+  multiply back), §3 "How LoRA and Quantization Fit Together" (two codes per byte, a
+  16-entry codebook, blocks with a scale each, dequantize to BF16 for compute, base +
+  adapter), §4 "One QLoRA Training Step, End to End" (gradients reach the adapters, the
+  base is never updated), §5 "NF4" (levels at quantiles of a standard normal), §6 "Double
+  Quantization Compresses the Scales" (quantize the block scales; codes unchanged).
+* "QLoRA: Efficient Finetuning of Quantized LLMs" (mchromiak.github.io): "The algebra"
+  (X is t x h, W is h x o, L1 is h x r, L2 is r x o, scalar s), "1. NormalFloat" (blocks
+  with their own scale, BF16 compute), "2. Double quantization" (8-bit first-level scales,
+  higher-precision second-level scales; 0.5 -> ~0.127 bits per weight), "A worked memory
+  budget for 65 billion weights" (64 weights per block, 256 scales per second-level block).
+* "QLoRA: the paper that put large-model fine-tuning on a desk" (goodomens.studio):
+  "Idea one: NF4" (each level used equally often), "Idea two: double quantization" (fp32
+  scale per 64 weights, re-quantized to 8 bits with a second-level scale per chunk), "The
+  core move" (a 4-bit block is dequantized on the fly, used for the matmul, discarded).
+* "Chapter 1: What is QLoRA?" (docs.skillversehub.com): "Key Components" (equal number of
+  values in each bin).
+
+Readings where the pages are silent (each is also listed in the design notes):
+
+* Codebook construction. The pages fix: quantiles of N(0,1), equal use of every level,
+  an exact zero, ends normalised to -1 and +1. The plainest construction with all four:
+  8 positive quantiles at probabilities evenly spaced from delta down to (not including)
+  1/2, 7 negative ones likewise, the zero, all divided by the largest; delta is the mean of
+  the two "centre of the outermost of 15 / of 16 equal-probability bins" probabilities,
+  1 - 1/30 and 1 - 1/32. The exact delta is a reading: parity of the 16 values is pinned
+  by the properties above, not by a printed table (the pages print none).
+* Code choice: nearest level by comparison against fp32 midpoints of adjacent levels; a
+  value exactly on a midpoint takes the lower code.
+* Second level: unsigned 8-bit absmax codes with step c2/255 (the textbook scheme of
+  "QLoRA in LLMs" §2 made unsigned because a block absmax is never negative, §1 on UINT8),
+  one fp32 scale per 256 first-level scales; the last group may be partial.
+* Layout: the stored matrix is Wt = W' transposed (o x h, row-major, "out x in"); blocks
+  of 64 run along h inside one row; element 2j of the flat order sits in the high nibble
+  of byte j.
+* LoRA: Y = X.W + s.X.L1.L2 with s = alpha / r; backward by the chain rule.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+BLOCK = 64          # weights per first-level block
+GROUP = 256         # first-level scales per second-level scale
+ZERO_CODE = 7       # index of the exact-zero level
+Q8_MAX = 255        # unsigned 8-bit code range for the first-level scales
+
+
+# ----------------------------------------------------------------------------------------
+# Standard normal quantile, by bisection on the CDF (double precision)
+# ----------------------------------------------------------------------------------------
+
+def normal_cdf(x: float) -> float:
+    """Phi(x) of the standard normal, from the complementary error function."""
+    return 0.5 * math.erfc(-x / math.sqrt(2.0))
+
+
+def normal_quantile(p: float) -> float:
+    """Phi^-1(p) by bisection: the x with Phi(x) = p, to the resolution of a double."""
+    if not 0.0 < p < 1.0:
+        raise ValueError("p must lie in (0, 1)")
+    lo, hi = -40.0, 40.0
+    for _ in range(2000):
+        mid = 0.5 * (lo + hi)
+        if mid == lo or mid == hi:
+            break
+        if normal_cdf(mid) < p:
+            lo = mid
+        else:
+            hi = mid
+    return 0.5 * (lo + hi)
+
+
+# ----------------------------------------------------------------------------------------
+# NF4 codebook ("QLoRA in LLMs" §5; "Idea one: NF4"; "Key Components")
+# ----------------------------------------------------------------------------------------
+
+def nf4_tail_probability() -> float:
+    """delta: mean of the centre probabilities of the outermost of 15 and of 16 equal bins."""
+    return 0.5 * ((1.0 - 1.0 / 30.0) + (1.0 - 1.0 / 32.0))
+
+
+def nf4_construction_probabilities() -> tuple[list[float], list[float]]:
+    """Probabilities at which the positive (8) and negative (7) levels are placed.
+
+    Positive side: delta + i*(1/2 - delta)/8 for i = 0..7 (the point 1/2 itself, i = 8, is
+    dropped; the zero level takes its place). Negative side: the same with 7 steps, i = 0..6,
+    mirrored (level = -Phi^-1(p)).
+    """
+    delta = nf4_tail_probability()
+    pos = [delta + i * (0.5 - delta) / 8.0 for i in range(8)]
+    neg = [delta + i * (0.5 - delta) / 7.0 for i in range(7)]
+    return pos, neg
+
+
+def nf4_codebook_f64() -> np.ndarray:
+    """The 16 levels in double precision, ascending, ends exactly -1 and +1, q[7] == 0."""
+    pos_p, neg_p = nf4_construction_probabilities()
+    pos = [normal_quantile(p) for p in pos_p]
+    neg = [-normal_quantile(p) for p in neg_p]
+    top = normal_quantile(nf4_tail_probability())
+    values = sorted(pos + neg + [0.0])
+    return np.array([v / top for v in values], dtype=np.float64)
+
+
+def nf4_codebook() -> np.ndarray:
+    """The 16 NF4 levels rounded to fp32 (the table the method stores and uses)."""
+    return nf4_codebook_f64().astype(np.float32)
+
+
+def nf4_midpoints(levels: np.ndarray | None = None) -> np.ndarray:
+    """15 fp32 decision thresholds m[i] = (q[i] + q[i+1]) / 2, summed in double."""
+    q = nf4_codebook() if levels is None else np.asarray(levels, dtype=np.float32)
+    q64 = q.astype(np.float64)
+    return ((q64[:-1] + q64[1:]) / 2.0).astype(np.float32)
+
+
+# ----------------------------------------------------------------------------------------
+# bf16 round-to-nearest-even ("QLoRA in LLMs" §1: BF16 = 8 exponent, 7 fraction bits)
+# ----------------------------------------------------------------------------------------
+
+def bf16_bits_rne(x: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 bit patterns (uint16), round to nearest, ties to even; NaN stays NaN."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    rounded = ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
+    nan = np.isnan(x)
+    if nan.any():
+        rounded = np.where(nan, ((u >> 16) | 0x40).astype(np.uint16), rounded)
+    return rounded
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> the fp32 values they stand for (exact)."""
+    b = np.ascontiguousarray(b, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """fp32 values rounded to the nearest bf16 value, returned as fp32."""
+    return bf16_bits_to_f32(bf16_bits_rne(x))
+
+
+# ----------------------------------------------------------------------------------------
+# Textbook absmax integer quantization ("QLoRA in LLMs" §2 "Choose a scale, then round")
+# ----------------------------------------------------------------------------------------
+
+def absmax_int_quantize(x: np.ndarray, qmax: int, signed: bool):
+    """Symmetric absmax quantization of one group to integers in [-qmax, qmax] (or [0, qmax]).
+
+    scale = max|x| / qmax (fp32); code = round-half-even(x / scale), clamped. Returns
+    (codes int64, scale fp32). An all-zero group has scale 0 and codes 0.
+    """
+    x = np.asarray(x, dtype=np.float32)
+    absmax = np.float32(np.max(np.abs(x))) if x.size else np.float32(0.0)
+    scale = np.float32(absmax / np.float32(qmax))
+    if scale == 0.0:
+        return np.zeros(x.shape, dtype=np.int64), scale
+    codes = np.rint(x / scale).astype(np.int64)
+    lo = -qmax if signed else 0
+    return np.clip(codes, lo, qmax), scale
+
+
+def absmax_int_dequantize(codes: np.ndarray, scale: np.float32) -> np.ndarray:
+    """Multiply the stored integers back by the group scale (fp32)."""
+    return np.asarray(codes, dtype=np.float32) * np.float32(scale)
+
+
+# ----------------------------------------------------------------------------------------
+# NF4 quantizer with double-quantized scales
+# ----------------------------------------------------------------------------------------
+
+class NF4Packed:
+    """The packed weight: codes (uint8, n/2), absmax_q8 (uint8, n/64), absmax_s2 (fp32)."""
+
+    def __init__(self, codes, absmax_q8, absmax_s2, out_features, in_features, absmax_f32):
+        self.codes = codes
+        self.absmax_q8 = absmax_q8
+        self.absmax_s2 = absmax_s2
+        self.out_features = out_features
+        self.in_features = in_features
+        self.absmax_f32 = absmax_f32       # first-level scales before double quantization
+
+
+def block_absmax(Wt: np.ndarray) -> np.ndarray:
+    """c1[b] = max |w| over block b (64 consecutive weights of the flat row-major order)."""
+    w = np.asarray(Wt, dtype=np.float32).reshape(-1, BLOCK)
+    return np.max(np.abs(w), axis=1)
+
+
+def nf4_codes(Wt: np.ndarray, levels: np.ndarray | None = None) -> np.ndarray:
+    """Unpacked 4-bit codes (uint8, one per weight) from the exact fp32 block absmax.
+
+    x_hat = w / c1 in fp32 (IEEE, round to nearest); code = number of midpoints strictly
+    below x_hat. A block whose absmax is 0 takes the zero level everywhere.
+    """
+    mid = nf4_midpoints(levels)
+    w = np.asarray(Wt, dtype=np.float32).reshape(-1, BLOCK)
+    c1 = np.max(np.abs(w), axis=1)
+    zero = c1 == 0
+    safe = np.where(zero, np.float32(1.0), c1).astype(np.float32)
+    xhat = (w / safe[:, None]).astype(np.float32)
+    codes = np.zeros(w.shape, dtype=np.uint8)
+    for i in range(mid.size):
+        codes += (xhat > mid[i]).astype(np.uint8)
+    codes[zero, :] = ZERO_CODE
+    return codes.reshape(-1)
+
+
+def pack_nibbles(codes: np.ndarray) -> np.ndarray:
+    """Two codes per byte: byte j = (code[2j] << 4) | code[2j+1]."""
+    c = np.asarray(codes, dtype=np.uint8).reshape(-1, 2)
+    return ((c[:, 0] << 4) | c[:, 1]).astype(np.uint8)
+
+
+def unpack_nibbles(packed: np.ndarray) -> np.ndarray:
+    """Inverse of pack_nibbles."""
+    p = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(p.size * 2, dtype=np.uint8)
+    out[0::2] = p >> 4
+    out[1::2] = p & 0xF
+    return out
+
+
+def double_quantize(c1: np.ndarray):
+    """Second-level quantization of the first-level scales.
+
+    Groups of 256 consecutive scales (the last one may be shorter): c2 = max c1,
+    s2 = c2 / 255 (fp32), q8 = clamp(round-half-even(c1 / s2), 0, 255). A group whose
+    maximum is 0 stores s2 = 0 and q8 = 0.
+    """
+    c1 = np.asarray(c1, dtype=np.float32)
+    nb = c1.size
+    ng = (nb + GROUP - 1) // GROUP
+    q8 = np.zeros(nb, dtype=np.uint8)
+    s2 = np.zeros(ng, dtype=np.float32)
+    for g in range(ng):
+        seg = c1[g * GROUP:(g + 1) * GROUP]
+        c2 = np.float32(np.max(seg))
+        scale = np.float32(c2 / np.float32(Q8_MAX))
+        s2[g] = scale
+        if scale == 0.0:
+            continue
+        ratio = (seg / scale).astype(np.float32)
+        q8[g * GROUP:(g + 1) * GROUP] = np.clip(np.rint(ratio), 0, Q8_MAX).astype(np.uint8)
+    return q8, s2
+
+
+def nf4_quantize(Wt: np.ndarray) -> NF4Packed:
+    """Quantize an fp32 weight stored as Wt (o x h, row-major, h % 64 == 0).
+
+    Raises ValueError for non-finite input (the library reports a status instead).
+    """
+    Wt = np.asarray(Wt, dtype=np.float32)
+    if Wt.ndim != 2 or Wt.shape[1] % BLOCK != 0:
+        raise ValueError("Wt must be o x h with h a multiple of 64")
+    if not np.all(np.isfinite(Wt)):
+        raise ValueError("non-finite weight")
+    c1 = block_absmax(Wt)
+    codes = nf4_codes(Wt)
+    q8, s2 = double_quantize(c1)
+    return NF4Packed(pack_nibbles(codes), q8, s2, Wt.shape[0], Wt.shape[1], c1)
+
+
+def block_scales(q8: np.ndarray, s2: np.ndarray) -> np.ndarray:
+    """Reconstructed first-level scale per block: float(q8[b]) * s2[b // 256] (fp32)."""
+    q8 = np.asarray(q8, dtype=np.uint8)
+    g = np.arange(q8.size) // GROUP
+    return (q8.astype(np.float32) * np.asarray(s2, dtype=np.float32)[g]).astype(np.float32)
+
+
+def nf4_dequantize_f32(packed: NF4Packed, levels: np.ndarray | None = None) -> np.ndarray:
+    """w' before the bf16 rounding: q[code] * (float(q8) * s2), two fp32 multiplies."""
+    q = nf4_codebook() if levels is None else np.asarray(levels, dtype=np.float32)
+    codes = unpack_nibbles(packed.codes).reshape(-1, BLOCK)
+    k = block_scales(packed.absmax_q8, packed.absmax_s2)
+    w = (q[codes] * k[:, None]).astype(np.float32)
+    return w.reshape(packed.out_features, packed.in_features)
+
+
+def nf4_dequantize_bits(packed: NF4Packed) -> np.ndarray:
+    """The dequantized weight as bf16 bit patterns (uint16, o x h)."""
+    return bf16_bits_rne(nf4_dequantize_f32(packed))
+
+
+def nf4_dequantize(packed: NF4Packed) -> np.ndarray:
+    """The dequantized weight W' (stored orientation o x h) as fp32 values of bf16 numbers."""
+    return bf16_bits_to_f32(nf4_dequantize_bits(packed))
+
+
+def dequantize_without_double_quant(codes: np.ndarray, c1: np.ndarray, o: int, h: int):
+    """w' with the exact fp32 block absmax (double quantization off), rounded to bf16."""
+    q = nf4_codebook()
+    c = np.asarray(codes, dtype=np.uint8).reshape(-1, BLOCK)
+    w = (q[c] * np.asarray(c1, dtype=np.float32)[:, None]).astype(np.float32)
+    return bf16_round(w.reshape(o, h))
+
+
+# ----------------------------------------------------------------------------------------
+# Storage ledger ("A worked memory budget for 65 billion weights"; "2. Double quantization")
+# ----------------------------------------------------------------------------------------
+
+def scale_bits_per_weight(double_quant: bool) -> float:
+    """Bits of scale metadata per weight: 32/64 without, 8/64 + 32/(64*256) with DQ."""
+    if not double_quant:
+        return 32.0 / BLOCK
+    return 8.0 / BLOCK + 32.0 / (BLOCK * GROUP)
+
+
+def packed_bytes(n: int) -> int:
+    """Bytes of the real packed format for n weights (n % 64 == 0)."""
+    nb = n // BLOCK
+    return n // 2 + nb + 4 * ((nb + GROUP - 1) // GROUP)
+
+
+def weight_storage_bytes(n_params: float, bits: float) -> float:
+    """Raw storage of n_params values at `bits` bits each (N * b / 8)."""
+    return n_params * bits / 8.0
+
+
+# ----------------------------------------------------------------------------------------
+# The adapted linear layer ("The algebra"; "QLoRA in LLMs" §3-§4)
+# ----------------------------------------------------------------------------------------
+
+def _f64(a) -> np.ndarray:
+    return np.asarray(a, dtype=np.float64)
+
+
+def qlora_linear_fwd(X, Wdq, L1, L2, s):
+    """Y = X.W' + s.(X.L1).L2 in fp64.
+
+    X: t x h; Wdq: the dequantized weight in its stored orientation o x h (so W' = Wdq^T,
+    h x o); L1: h x r; L2: r x o. Returns (Y t x o, sT = s.X.L1 t x r), both fp64.
+    """
+    X, Wt, L1, L2 = _f64(X), _f64(Wdq), _f64(L1), _f64(L2)
+    T = X @ L1
+    Y = X @ Wt.T + s * (T @ L2)
+    return Y, s * T
+
+
+def qlora_linear_bwd(dY, X, Wdq, L1, L2, s):
+    """Gradients of <dY, Y> for Y = X.W' + s.X.L1.L2, in fp64. W' gets none.
+
+    dX = dY.W'^T + s.(dY.L2^T).L1^T; dL1 = s.X^T.(dY.L2^T); dL2 = s.(X.L1)^T.dY.
+    Returns (dX t x h, dL1 h x r, dL2 r x o, sU = s.dY.L2^T t x r).
+    """
+    dY, X, Wt, L1, L2 = _f64(dY), _f64(X), _f64(Wdq), _f64(L1), _f64(L2)
+    U = dY @ L2.T
+    dX = dY @ Wt + s * (U @ L1.T)
+    dL1 = s * (X.T @ U)
+    dL2 = s * ((X @ L1).T @ dY)
+    return dX, dL1, dL2, s * U
+
+
+def qlora_linear_fwd_rows(rows, X, Wdq, L1, L2, s):
+    """Rows `rows` of Y only (each row of Y depends on the same row of X alone)."""
+    rows = np.asarray(rows)
+    Y, _ = qlora_linear_fwd(_f64(X)[rows], Wdq, L1, L2, s)
+    return Y
+
+
+def qlora_linear_bwd_dx_rows(rows, dY, Wdq, L1, L2, s):
+    """Rows `rows` of dX only (each row of dX depends on the same row of dY alone)."""
+    dY, Wt, L1, L2 = _f64(dY)[np.asarray(rows)], _f64(Wdq), _f64(L1), _f64(L2)
+    return dY @ Wt + s * ((dY @ L2.T) @ L1.T)
+
+
+def max_err_vs_rms(got, ref) -> tuple[float, float]:
+    """(max |got - ref|, RMS(ref)) in fp64: the tolerance test is max <= 2e-2 * RMS."""
+    got, ref = _f64(got), _f64(ref)
+    return float(np.max(np.abs(got - ref))) if ref.size else 0.0, \
+        float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
