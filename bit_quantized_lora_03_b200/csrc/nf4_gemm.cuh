@@ -1,0 +1,461 @@
+// tcgen05 (5th-generation tensor core) GEMMs for the training-shape QLoRA linear on sm_100a.
+//
+// 1) nf4_gemm_kernel<BWD>: the frozen-base product with the NF4 dequantization fused into the
+//    producer stage and the LoRA product folded into the same TMEM accumulator:
+//       forward  (BWD = false):  Y  = X  . W'   + sT . L2      (M = t, N = o, K = h)
+//       backward (BWD = true):   dX = dY . W'^T + sU . L1^T    (M = t, N = h, K = o)
+//    ("The algebra", mchromiak.github.io; "QLoRA in LLMs" sections 3-4; "The core move",
+//    goodomens.studio: each 4-bit block is dequantized on the fly, used, discarded.)
+//    A (X or dY) and the packed codes arrive by TMA; 8 producer warps turn each 64-weight
+//    block into bf16 (w' = bf16(level * (q8 * s2)), the exact nf4_dequantize values) and
+//    write it straight into the 128-byte-swizzled operand layout the MMA reads: K-major for
+//    the forward (rows of Wt are N), MN-major for the backward (rows of Wt are K). One thread
+//    issues tcgen05.mma into a 128 x 256 fp32 accumulator in tensor memory; the r/64 LoRA
+//    K-steps (A = sT or sU, B = L2 or L1, both by TMA) run first, then the h/64 (or o/64)
+//    weight K-steps. Four epilogue warps read TMEM and write bf16.
+//
+// 2) tc_gemm_kernel<A_MN, B_MN>: a plain TMA-fed tcgen05 GEMM (both operands by TMA, either
+//    major-ness) with split-K and fp32 atomic or bf16 output, for the rank-r products
+//    T = X.L1, U = dY.L2^T, dL1 = X^T.sU and dL2^T = dY^T.sT.
+//
+// Every wait is bounded (qlora::mbar_wait); on expiry the CTA reports QLORA_DEV_TIMEOUT,
+// stops issuing, waits for its own copies and MMAs in flight, frees TMEM and returns.
+#pragma once
+
+#include "nf4_codec.cuh"
+
+namespace qlora {
+namespace tc {
+
+constexpr int BM = 128;        // tokens per tile (TMEM lanes)
+constexpr int BN = 256;        // output columns per tile (TMEM fp32 columns)
+constexpr int BK = 64;         // K per stage: one 128-byte swizzle row of bf16, one NF4 block
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;       // 16 KB
+constexpr int B_BYTES = BN * BK * 2;       // 32 KB
+constexpr int P_BYTES = BN * BK / 2;       // 8 KB of packed codes
+constexpr int kEpiWarps = 4;               // warps 0-3: epilogue (TMEM lanes 0-127)
+constexpr int kDeqWarps = 8;               // warps 4-11: dequant producers
+constexpr int kTmaWarp = 12;
+constexpr int kMmaWarp = 13;
+constexpr int kThreads = 14 * 32;
+constexpr int kTmemCols = 256;
+
+constexpr size_t nf4_gemm_smem_bytes() {
+  return 1024 /* alignment slack */ + STAGES * (A_BYTES + B_BYTES + P_BYTES) + 256;
+}
+
+}  // namespace tc
+
+struct Nf4GemmArgs {
+  const uint8_t* q8;
+  const float* s2;
+  int64_t h;        // in_features: row length of Wt
+  int M;            // tokens
+  int N;            // output columns: o (forward) or h (backward)
+  int num_kb;       // weight K-steps: h/64 (forward) or o/64 (backward)
+  int num_lkb;      // LoRA K-steps: ceil(r/64)
+  uint16_t* out;    // M x N bf16, row stride N
+  Nf4Table tab;
+};
+
+// Wait for an mbarrier phase ignoring the abort flag (used only to drain in-flight copies
+// after an abort), still bounded by the timeout.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      report(kDevTimeout);
+      return;
+    }
+  }
+}
+
+template <bool kBwd>
+__global__ void __launch_bounds__(tc::kThreads, 1)
+    nf4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmP,
+                    const __grid_constant__ CUtensorMap tmA2,
+                    const __grid_constant__ CUtensorMap tmB2, const Nf4GemmArgs args) {
+  using namespace tc;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + STAGES * A_BYTES;
+  uint8_t* sP = sB + STAGES * B_BYTES;
+  uint64_t* full_ap = reinterpret_cast<uint64_t*>(sP + STAGES * P_BYTES);
+  uint64_t* full_b = full_ap + STAGES;
+  uint64_t* empty = full_b + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
+  volatile uint32_t* abort_flag = tmem_holder + 1;
+  float* lv = reinterpret_cast<float*>(tmem_holder + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * BN;
+  const int m0 = blockIdx.y * BM;
+  const int total = args.num_lkb + args.num_kb;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_ap[s], 1);
+      mbar_init(&full_b[s], kDeqWarps * 32);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (threadIdx.x < 16) lv[threadIdx.x] = args.tab.level[threadIdx.x];
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_holder, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == kTmaWarp && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmP);
+    tma_prefetch_desc(&tmA2);
+    tma_prefetch_desc(&tmB2);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == kTmaWarp) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < total; ++i) {
+        const int slot = i % STAGES;
+        const uint32_t ph = (i / STAGES) & 1;
+        if (!mbar_wait(&empty[slot], ph ^ 1u, abort_flag)) break;
+        uint8_t* a_dst = sA + slot * A_BYTES;
+        if (i < args.num_lkb) {
+          mbar_arrive_expect_tx(&full_ap[slot], A_BYTES + B_BYTES);
+          tma_load_2d(a_dst, &tmA2, &full_ap[slot], i * BK, m0);
+          if (!kBwd) {
+            // L2 (r x o), MN-major B: four 64-column atoms, 8 KB apart
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+              tma_load_2d(sB + slot * B_BYTES + a * 8192, &tmB2, &full_ap[slot], n0 + a * 64,
+                          i * BK);
+          } else {
+            // L1 (h x r), K-major B: 256 rows of 64 ranks
+            tma_load_2d(sB + slot * B_BYTES, &tmB2, &full_ap[slot], i * BK, n0);
+          }
+        } else {
+          const int kb = i - args.num_lkb;
+          mbar_arrive_expect_tx(&full_ap[slot], A_BYTES + P_BYTES);
+          tma_load_2d(a_dst, &tmA, &full_ap[slot], kb * BK, m0);
+          if (!kBwd) {
+            tma_load_2d(sP + slot * P_BYTES, &tmP, &full_ap[slot], kb * (BK / 2), n0);
+          } else {
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+              tma_load_2d(sP + slot * P_BYTES + a * 2048, &tmP, &full_ap[slot], n0 / 2 + a * 32,
+                          kb * BK);
+          }
+        }
+        issued = i + 1;
+      }
+      if (*abort_flag) {
+        // make sure no copy is still writing this CTA's shared memory before it exits
+        for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
+          mbar_drain(&full_ap[j % STAGES], (j / STAGES) & 1);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t kIdescMain = idesc_bf16(BM, BN, false, kBwd);
+      constexpr uint32_t kIdescLora = idesc_bf16(BM, BN, false, !kBwd);
+      bool any = false;
+      for (int i = 0; i < total; ++i) {
+        const int slot = i % STAGES;
+        const uint32_t ph = (i / STAGES) & 1;
+        if (!mbar_wait(&full_ap[slot], ph, abort_flag)) break;
+        if (!mbar_wait(&full_b[slot], ph, abort_flag)) break;
+        tc_fence_after();
+        const bool lora = i < args.num_lkb;
+        const bool b_mn = lora ? !kBwd : kBwd;
+        const uint32_t idesc = lora ? kIdescLora : kIdescMain;
+        const uint32_t a_addr = smem_addr(sA + slot * A_BYTES);
+        const uint32_t b_addr = smem_addr(sB + slot * B_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          const uint64_t ad = sw128_desc(a_addr + kk * 32, 16, 1024);
+          const uint64_t bd = b_mn ? sw128_desc(b_addr + kk * 2048, 8192, 1024)
+                                   : sw128_desc(b_addr + kk * 32, 16, 1024);
+          umma_bf16(tmem_base, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&empty[slot]);
+        any = true;
+      }
+      // completes once every MMA above has finished (also after an abort)
+      umma_commit(acc_full);
+      if (*abort_flag && any) mbar_drain(acc_full, 0);
+    }
+  } else if (warp >= kEpiWarps && warp < kEpiWarps + kDeqWarps) {
+    // ---------------- dequant producers: one 64-weight block per thread per stage ----------
+    const int p = threadIdx.x - kEpiWarps * 32;  // 0..255
+    const int64_t nblk_row = args.h / kBlock;
+    int64_t qidx_base;
+    int out_off;
+    int pk_off;
+    bool valid;
+    if (!kBwd) {
+      // row p of the N tile is Wt row n0 + p; its block kb is K-step kb
+      const int64_t j = n0 + p;
+      valid = j < args.N;
+      qidx_base = j * nblk_row;
+      pk_off = p * 32;
+      out_off = (p >> 3) * 1024 + (p & 7) * 128;
+    } else {
+      // K row jl of the stage is Wt row kb*64 + jl; column atom a is blocks n0/64 + a
+      const int jl = p & 63, a = p >> 6;
+      valid = (n0 + a * 64) < args.N;
+      qidx_base = (n0 / 64) + a;
+      pk_off = a * 2048 + jl * 32;
+      out_off = a * 8192 + (jl >> 3) * 1024 + (jl & 7) * 128;
+    }
+    const int swz = (!kBwd ? p : (p & 63)) & 7;
+    for (int i = 0; i < total; ++i) {
+      const int slot = i % STAGES;
+      const uint32_t ph = (i / STAGES) & 1;
+      float k = 0.f;
+      if (i >= args.num_lkb && valid) {
+        const int kb = i - args.num_lkb;
+        const int64_t qi = !kBwd ? qidx_base + kb
+                                 : (static_cast<int64_t>(kb) * 64 + (p & 63)) * nblk_row + qidx_base;
+        k = __fmul_rn(static_cast<float>(__ldg(args.q8 + qi)), __ldg(args.s2 + (qi >> 8)));
+      }
+      if (!mbar_wait(&empty[slot], ph ^ 1u, abort_flag)) break;
+      if (i >= args.num_lkb) {
+        if (!mbar_wait(&full_ap[slot], ph, abort_flag)) break;
+        if (valid) {
+          const uint4* src = reinterpret_cast<const uint4*>(sP + slot * P_BYTES + pk_off);
+          const uint4 c0 = src[0], c1 = src[1];
+          const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          uint8_t* dst = sB + slot * B_BYTES + out_off;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t x = words[c];
+            uint4 o;
+            o.x = pack_bf16x2(__fmul_rn(lv[(x >> 4) & 15u], k), __fmul_rn(lv[x & 15u], k));
+            o.y = pack_bf16x2(__fmul_rn(lv[(x >> 12) & 15u], k), __fmul_rn(lv[(x >> 8) & 15u], k));
+            o.z = pack_bf16x2(__fmul_rn(lv[(x >> 20) & 15u], k), __fmul_rn(lv[(x >> 16) & 15u], k));
+            o.w = pack_bf16x2(__fmul_rn(lv[(x >> 28) & 15u], k), __fmul_rn(lv[(x >> 24) & 15u], k));
+            *reinterpret_cast<uint4*>(dst + ((c ^ swz) << 4)) = o;
+          }
+        }
+        fence_proxy_async_smem();
+      }
+      mbar_arrive(&full_b[slot]);
+    }
+  } else if (warp < kEpiWarps) {
+    // ---------------- epilogue: TMEM -> registers -> bf16 -> global -------------------------
+    const bool ok = mbar_wait(acc_full, 0, abort_flag);
+    tc_fence_after();
+    if (ok && !*abort_flag) {
+      const int row = m0 + warp * 32 + lane;
+      const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+      for (int c = 0; c < BN / 16; ++c) {
+        if (n0 + c * 16 >= args.N) break;  // N is a multiple of 64: whole chunks only
+        uint32_t v[16];
+        tmem_ld_16(lane_addr + c * 16, v);
+        tmem_ld_wait();
+        if (row < args.M) {
+          uint4 o0, o1;
+          o0.x = pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1]));
+          o0.y = pack_bf16x2(__uint_as_float(v[2]), __uint_as_float(v[3]));
+          o0.z = pack_bf16x2(__uint_as_float(v[4]), __uint_as_float(v[5]));
+          o0.w = pack_bf16x2(__uint_as_float(v[6]), __uint_as_float(v[7]));
+          o1.x = pack_bf16x2(__uint_as_float(v[8]), __uint_as_float(v[9]));
+          o1.y = pack_bf16x2(__uint_as_float(v[10]), __uint_as_float(v[11]));
+          o1.z = pack_bf16x2(__uint_as_float(v[12]), __uint_as_float(v[13]));
+          o1.w = pack_bf16x2(__uint_as_float(v[14]), __uint_as_float(v[15]));
+          uint4* dst = reinterpret_cast<uint4*>(args.out + static_cast<int64_t>(row) * args.N +
+                                                n0 + c * 16);
+          dst[0] = o0;
+          dst[1] = o1;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Plain TMA-fed tcgen05 GEMM for the rank-r products.
+// D (M x Ncols) = alpha * A (M x K) . B (K x Ncols), Ncols <= 256 (one N tile), split-K over
+// blockIdx.z. A_MN / B_MN select MN-major operands (the TMA boxes are 64 x 64 atoms then).
+// ------------------------------------------------------------------------------------------
+namespace tcg {
+constexpr int BM = 128, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;        // 16 KB
+constexpr int B_MAX_BYTES = 256 * BK * 2;   // 32 KB
+constexpr int kThreads = 6 * 32;            // warps 0-3 epilogue, 4 TMA, 5 MMA
+constexpr int kTmaWarp = 4, kMmaWarp = 5;
+constexpr size_t smem_bytes() { return 1024 + STAGES * (A_BYTES + B_MAX_BYTES) + 256; }
+}  // namespace tcg
+
+enum TcOutMode : int {
+  kOutAtomicRowMajor = 0,   // out32[m * ld + n] += alpha * acc
+  kOutAtomicTransposed = 1, // out32[n * ld + m] += alpha * acc
+};
+
+struct TcGemmArgs {
+  int M;
+  int Ncols;         // real number of output columns (<= BNp)
+  int BNp;           // MMA N: Ncols rounded up to a multiple of 16
+  int num_kb;        // ceil(K / 64)
+  int kb_per_split;
+  float alpha;
+  int out_mode;
+  float* out32;
+  int64_t ld;
+};
+
+template <bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(tcg::kThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const TcGemmArgs args) {
+  using namespace tcg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + STAGES * A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_MAX_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
+  volatile uint32_t* abort_flag = tmem_holder + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * BM;
+  const int kb0 = blockIdx.z * args.kb_per_split;
+  const int kb1 = min(args.num_kb, kb0 + args.kb_per_split);
+  const int nk = kb1 - kb0;
+  const int BNp = args.BNp;
+  const uint32_t tmem_cols = BNp <= 32 ? 32u : (BNp <= 64 ? 64u : (BNp <= 128 ? 128u : 256u));
+  const int b_atoms = (BNp + 63) / 64;
+  const uint32_t b_bytes = B_MN ? static_cast<uint32_t>(b_atoms) * 8192u
+                                : static_cast<uint32_t>(BNp) * 128u;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_holder, tmem_cols);
+    tmem_relinquish();
+  }
+  if (warp == kTmaWarp && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == kTmaWarp) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < nk; ++i) {
+        const int slot = i % STAGES;
+        const uint32_t ph = (i / STAGES) & 1;
+        if (!mbar_wait(&empty[slot], ph ^ 1u, abort_flag)) break;
+        const int kb = kb0 + i;
+        mbar_arrive_expect_tx(&full[slot], A_BYTES + b_bytes);
+        uint8_t* a_dst = sA + slot * A_BYTES;
+        if (!A_MN) {
+          tma_load_2d(a_dst, &tmA, &full[slot], kb * BK, m0);
+        } else {
+          tma_load_2d(a_dst, &tmA, &full[slot], m0, kb * BK);
+          tma_load_2d(a_dst + 8192, &tmA, &full[slot], m0 + 64, kb * BK);
+        }
+        uint8_t* b_dst = sB + slot * B_MAX_BYTES;
+        if (!B_MN) {
+          tma_load_2d(b_dst, &tmB, &full[slot], kb * BK, 0);
+        } else {
+          for (int a = 0; a < b_atoms; ++a)
+            tma_load_2d(b_dst + a * 8192, &tmB, &full[slot], a * 64, kb * BK);
+        }
+        issued = i + 1;
+      }
+      if (*abort_flag) {
+        for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
+          mbar_drain(&full[j % STAGES], (j / STAGES) & 1);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(BM, BNp, A_MN, B_MN);
+      bool any = false;
+      for (int i = 0; i < nk; ++i) {
+        const int slot = i % STAGES;
+        const uint32_t ph = (i / STAGES) & 1;
+        if (!mbar_wait(&full[slot], ph, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_addr(sA + slot * A_BYTES);
+        const uint32_t b_addr = smem_addr(sB + slot * B_MAX_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          const uint64_t ad = A_MN ? sw128_desc(a_addr + kk * 2048, 8192, 1024)
+                                   : sw128_desc(a_addr + kk * 32, 16, 1024);
+          const uint64_t bd = B_MN ? sw128_desc(b_addr + kk * 2048, 8192, 1024)
+                                   : sw128_desc(b_addr + kk * 32, 16, 1024);
+          umma_bf16(tmem_base, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&empty[slot]);
+        any = true;
+      }
+      umma_commit(acc_full);
+      if (*abort_flag && any) mbar_drain(acc_full, 0);
+    }
+  } else if (warp < 4) {
+    const bool ok = (nk > 0) && mbar_wait(acc_full, 0, abort_flag);
+    tc_fence_after();
+    if (ok && !*abort_flag) {
+      const int row = m0 + warp * 32 + lane;
+      const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+      for (int c = 0; c < BNp / 16; ++c) {
+        uint32_t v[16];
+        tmem_ld_16(lane_addr + c * 16, v);
+        tmem_ld_wait();
+        if (row < args.M) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int n = c * 16 + e;
+            if (n < args.Ncols) {
+              const float val = args.alpha * __uint_as_float(v[e]);
+              float* dst = args.out_mode == kOutAtomicRowMajor
+                               ? args.out32 + static_cast<int64_t>(row) * args.ld + n
+                               : args.out32 + static_cast<int64_t>(n) * args.ld + row;
+              atomicAdd(dst, val);
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, tmem_cols);
+  }
+}
+
+}  // namespace qlora

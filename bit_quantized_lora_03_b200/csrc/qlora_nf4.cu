@@ -1,0 +1,680 @@
+// libqlora_nf4: host implementation of the C ABI declared in include/qlora_nf4.h.
+//
+// Validates every argument on the host before any CUDA call, derives the NF4 codebook, builds
+// TMA tensor maps (cuTensorMapEncodeTiled through the runtime's driver entry point, so the
+// library does not link libcuda), and launches the hand-written sm_100a kernels of csrc/ on
+// the caller's stream. It never allocates device memory: scratch comes from the caller.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "qlora_nf4.h"
+
+#include "nf4_codec.cuh"
+#include "nf4_gemm.cuh"
+#include "nf4_gemv.cuh"
+
+using namespace qlora;
+
+namespace {
+
+// ------------------------------------------------------------------------------------------
+// NF4 codebook ("QLoRA in LLMs" section 5; "Idea one: NF4" on goodomens.studio; "Key
+// Components" on docs.skillversehub.com): 16 levels at standard-normal quantiles, an exact
+// zero, ends normalised to -1 and +1. Eight positive levels at probabilities evenly spaced
+// from delta towards 1/2 (1/2 itself excluded), seven negative ones likewise, plus zero, all
+// divided by the largest; delta = ((1 - 1/30) + (1 - 1/32)) / 2. Computed here in double
+// with a safeguarded Newton iteration on Phi(x) = p and rounded once to fp32.
+// ------------------------------------------------------------------------------------------
+double normal_cdf(double x) { return 0.5 * std::erfc(-x / std::sqrt(2.0)); }
+
+double normal_pdf(double x) { return std::exp(-0.5 * x * x) / std::sqrt(2.0 * 3.14159265358979323846); }
+
+double normal_quantile(double p) {
+  double lo = -40.0, hi = 40.0, x = 0.0;
+  for (int it = 0; it < 500; ++it) {
+    const double f = normal_cdf(x) - p;
+    if (f < 0.0) lo = x; else hi = x;
+    const double d = normal_pdf(x);
+    double xn = d > 0.0 ? x - f / d : 0.5 * (lo + hi);
+    if (!(xn > lo && xn < hi)) xn = 0.5 * (lo + hi);
+    if (xn == x) break;
+    x = xn;
+  }
+  return x;
+}
+
+struct Codebook {
+  float level[16];
+  float mid[15];
+};
+
+const Codebook& codebook() {
+  static Codebook cb = [] {
+    Codebook c{};
+    const double delta = 0.5 * ((1.0 - 1.0 / 30.0) + (1.0 - 1.0 / 32.0));
+    std::vector<double> v;
+    for (int i = 0; i < 8; ++i) v.push_back(normal_quantile(delta + i * (0.5 - delta) / 8.0));
+    for (int i = 0; i < 7; ++i) v.push_back(-normal_quantile(delta + i * (0.5 - delta) / 7.0));
+    v.push_back(0.0);
+    std::sort(v.begin(), v.end());
+    const double top = normal_quantile(delta);
+    for (int i = 0; i < 16; ++i) c.level[i] = static_cast<float>(v[i] / top);
+    for (int i = 0; i < 15; ++i)
+      c.mid[i] = static_cast<float>((static_cast<double>(c.level[i]) +
+                                     static_cast<double>(c.level[i + 1])) / 2.0);
+    return c;
+  }();
+  return cb;
+}
+
+Nf4Table device_table() {
+  Nf4Table t{};
+  const Codebook& cb = codebook();
+  for (int i = 0; i < 16; ++i) t.level[i] = cb.level[i];
+  for (int i = 0; i < 15; ++i) t.mid[i] = cb.mid[i];
+  t.mid[15] = 2.0f;
+  return t;
+}
+
+// ------------------------------------------------------------------------------------------
+// device checks, kernel attributes
+// ------------------------------------------------------------------------------------------
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  std::once_flag once;
+  int ok = 0;        // 1 = sm_100 device ready
+  int sms = 148;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+int current_device(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return QLORA_ERR_UNSUPPORTED_DEVICE;
+  DeviceInfo& d = g_dev[dev];
+  std::call_once(d.once, [&] {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      d.ok = -1;
+      return;
+    }
+    if (major != 10 || minor != 0) {
+      d.ok = -2;
+      return;
+    }
+    d.sms = sms;
+    bool fine = true;
+    fine &= cudaFuncSetAttribute(nf4_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(tc::nf4_gemm_smem_bytes())) == cudaSuccess;
+    fine &= cudaFuncSetAttribute(nf4_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(tc::nf4_gemm_smem_bytes())) == cudaSuccess;
+    fine &= cudaFuncSetAttribute(tc_gemm_kernel<false, false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(tcg::smem_bytes())) == cudaSuccess;
+    fine &= cudaFuncSetAttribute(tc_gemm_kernel<false, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(tcg::smem_bytes())) == cudaSuccess;
+    fine &= cudaFuncSetAttribute(tc_gemm_kernel<true, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(tcg::smem_bytes())) == cudaSuccess;
+    if (!fine) cudaGetLastError();
+    d.ok = fine ? 1 : -1;
+  });
+  *dev_out = dev;
+  if (d.ok == 1) return QLORA_OK;
+  return d.ok == -2 ? QLORA_ERR_UNSUPPORTED_DEVICE : QLORA_ERR_CUDA;
+}
+
+int sm_count(int dev) { return g_dev[dev].sms; }
+
+int launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------------------------------
+// kernel timing: CUDA events around each launch while a profile is open
+// ------------------------------------------------------------------------------------------
+namespace prof {
+enum Kind {
+  kQuant = 0, kDequant, kGemv, kGemvFinalize, kScaleRound, kTcGemm, kGemmFwd, kGemmBwd, kKinds
+};
+const char* const kNames[kKinds] = {
+    "nf4_quantize_kernel", "nf4_dequantize_kernel", "nf4_gemv_kernel",
+    "gemv_lora_finalize_kernel", "lora_scale_round_kernel", "tc_gemm_kernel",
+    "nf4_gemm_kernel<fwd>", "nf4_gemm_kernel<bwd>"};
+static_assert(kKinds == QLORA_KERNEL_KINDS, "kernel kinds");
+
+struct State {
+  std::mutex mu;
+  std::atomic<bool> on{false};
+  bool overflow = false;
+  std::vector<cudaEvent_t> events;  // two per record
+  std::vector<int> kinds;
+  int capacity = 0;
+  int n = 0;
+};
+State g;
+
+// Records a start event now and a stop event when it goes out of scope (after the launch).
+struct Scope {
+  int idx = -1;
+  cudaStream_t st;
+  Scope(int kind, cudaStream_t s) : st(s) {
+    if (!g.on.load(std::memory_order_relaxed)) return;
+    std::lock_guard<std::mutex> lock(g.mu);
+    if (!g.on.load()) return;
+    if (g.n >= g.capacity) {
+      g.overflow = true;
+      return;
+    }
+    idx = g.n++;
+    g.kinds[idx] = kind;
+    cudaEventRecord(g.events[2 * idx], st);
+  }
+  ~Scope() {
+    if (idx >= 0) cudaEventRecord(g.events[2 * idx + 1], st);
+  }
+};
+}  // namespace prof
+
+// ------------------------------------------------------------------------------------------
+// TMA tensor maps
+// ------------------------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      return static_cast<EncodeTiledFn>(nullptr);
+    }
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// 2-D map over a row-major matrix: `inner` contiguous elements per row, `outer` rows,
+// `row_bytes` between rows; box = box_inner x box_outer elements.
+bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                 uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                 bool swizzle128) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool map_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
+              uint32_t box_rows) {
+  return make_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, cols, rows, cols * 2, box_cols,
+                     box_rows, true);
+}
+
+// ------------------------------------------------------------------------------------------
+// argument checks
+// ------------------------------------------------------------------------------------------
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int64_t kMaxDim = int64_t(1) << 31;
+
+int check_weight(const nf4_weight* q) {
+  if (!q || !q->codes || !q->absmax_q8 || !q->absmax_s2) return QLORA_ERR_INVALID_ARG;
+  if (q->out_features < 1 || q->in_features < 64 || q->in_features % 64 != 0)
+    return QLORA_ERR_BAD_SHAPE;
+  if (q->out_features >= kMaxDim || q->in_features >= kMaxDim) return QLORA_ERR_BAD_SHAPE;
+  const int64_t n = q->out_features * q->in_features;
+  if (n / q->in_features != q->out_features || n > (int64_t(1) << 46)) return QLORA_ERR_BAD_SHAPE;
+  if (!aligned16(q->codes) || !aligned16(q->absmax_q8) || !aligned16(q->absmax_s2))
+    return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+int check_linear_shape(int64_t t, int64_t h, int64_t o, int64_t r) {
+  if (t < 1 || r < 16 || r > 256 || r % 16 != 0) return QLORA_ERR_INVALID_ARG;
+  if (h < 64 || h % 64 != 0 || o < 64 || o % 64 != 0) return QLORA_ERR_BAD_SHAPE;
+  if (t >= kMaxDim || h >= kMaxDim || o >= kMaxDim) return QLORA_ERR_BAD_SHAPE;
+  return QLORA_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// workspace regions (each 256-byte aligned): fp32 t x r accumulator, bf16 t x r
+size_t lora_region_bytes(int64_t t, int64_t r) {
+  return align256(static_cast<size_t>(t) * r * 4) + align256(static_cast<size_t>(t) * r * 2);
+}
+
+// fp32 t x o accumulator for the GEMV's split-K partial sums
+size_t gemv_region_bytes(int64_t t, int64_t o) {
+  return align256(static_cast<size_t>(t) * o * 4);
+}
+
+constexpr int64_t kGemvMaxTokens = 16;
+
+// ------------------------------------------------------------------------------------------
+// launch helpers
+// ------------------------------------------------------------------------------------------
+int splits_for(int ctas, int num_kb, int sms) {
+  int s = std::max(1, (sms + ctas - 1) / std::max(1, ctas));
+  s = std::min(s, num_kb);
+  return std::max(1, s);
+}
+
+// D (M x ncols) += alpha * A . B with the generic tcgen05 GEMM, split-K so the grid fills the
+// GPU. Output fp32 by atomic adds (caller zeroes it).
+template <bool A_MN, bool B_MN>
+int launch_tc_gemm(const CUtensorMap& mA, const CUtensorMap& mB, int64_t M, int64_t ncols,
+                   int64_t K, float alpha, int mode, float* out32, int64_t ld, int sms,
+                   cudaStream_t st) {
+  TcGemmArgs a{};
+  a.M = static_cast<int>(M);
+  a.Ncols = static_cast<int>(ncols);
+  a.BNp = static_cast<int>((ncols + 15) / 16 * 16);
+  a.num_kb = static_cast<int>((K + 63) / 64);
+  const int mtiles = static_cast<int>((M + 127) / 128);
+  const int splits = splits_for(mtiles, a.num_kb, sms);
+  a.kb_per_split = (a.num_kb + splits - 1) / splits;
+  const int zs = (a.num_kb + a.kb_per_split - 1) / a.kb_per_split;
+  a.alpha = alpha;
+  a.out_mode = mode;
+  a.out32 = out32;
+  a.ld = ld;
+  dim3 grid(1, mtiles, zs);
+  {
+    prof::Scope ps(prof::kTcGemm, st);
+    tc_gemm_kernel<A_MN, B_MN><<<grid, tcg::kThreads, tcg::smem_bytes(), st>>>(mA, mB, a);
+  }
+  return launch_status();
+}
+
+struct LoraWs {
+  float* acc32;   // t x r fp32
+  uint16_t* b16;  // t x r bf16
+};
+
+LoraWs carve_lora(void* base, int64_t t, int64_t r) {
+  LoraWs w;
+  w.acc32 = reinterpret_cast<float*>(base);
+  w.b16 = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(base) +
+                                      align256(static_cast<size_t>(t) * r * 4));
+  return w;
+}
+
+// s . A . B^(T) for the rank-r down projections: out16 = bf16(s * A.B) (and out16b if given).
+// A is t x K (K-major), B is given by its map. Uses ws.acc32 as the fp32 accumulator.
+template <bool B_MN>
+int lora_down(const CUtensorMap& mA, const CUtensorMap& mB, int64_t t, int64_t K, int64_t r,
+              float s, const LoraWs& ws, uint16_t* out16, uint16_t* out16b, int sms,
+              cudaStream_t st) {
+  if (cudaMemsetAsync(ws.acc32, 0, static_cast<size_t>(t) * r * 4, st) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  int rc = launch_tc_gemm<false, B_MN>(mA, mB, t, r, K, 1.0f, kOutAtomicRowMajor, ws.acc32, r,
+                                       sms, st);
+  if (rc) return rc;
+  const int64_t count = t * r;
+  {
+    prof::Scope ps(prof::kScaleRound, st);
+    lora_scale_round_kernel<<<static_cast<unsigned>((count + 255) / 256), 256, 0, st>>>(
+        ws.acc32, out16, out16b, count, s);
+  }
+  return launch_status();
+}
+
+}  // namespace
+
+// ==========================================================================================
+// C ABI
+// ==========================================================================================
+extern "C" {
+
+int qlora_nf4_codebook(float* levels, float* midpoints) {
+  if (!levels) return QLORA_ERR_INVALID_ARG;
+  const Codebook& cb = codebook();
+  std::memcpy(levels, cb.level, sizeof(cb.level));
+  if (midpoints) std::memcpy(midpoints, cb.mid, sizeof(cb.mid));
+  return QLORA_OK;
+}
+
+const char* qlora_status_string(int status) {
+  switch (status) {
+    case QLORA_OK: return "QLORA_OK";
+    case QLORA_ERR_INVALID_ARG: return "QLORA_ERR_INVALID_ARG: null pointer or invalid argument";
+    case QLORA_ERR_BAD_SHAPE: return "QLORA_ERR_BAD_SHAPE: unsupported shape";
+    case QLORA_ERR_MISALIGNED: return "QLORA_ERR_MISALIGNED: pointer not 16-byte aligned";
+    case QLORA_ERR_WORKSPACE: return "QLORA_ERR_WORKSPACE: workspace missing or too small";
+    case QLORA_ERR_CUDA: return "QLORA_ERR_CUDA: CUDA runtime or launch error";
+    case QLORA_ERR_UNSUPPORTED_DEVICE: return "QLORA_ERR_UNSUPPORTED_DEVICE: not an sm_100 GPU";
+    case QLORA_DEV_NONFINITE: return "QLORA_DEV_NONFINITE: non-finite weight";
+    case QLORA_DEV_TIMEOUT: return "QLORA_DEV_TIMEOUT: a kernel wait timed out";
+    case QLORA_DEV_NONFINITE | QLORA_DEV_TIMEOUT:
+      return "QLORA_DEV_NONFINITE|QLORA_DEV_TIMEOUT";
+    default: return "unknown status";
+  }
+}
+
+size_t qlora_fwd_workspace_bytes(int64_t t, int64_t h, int64_t o, int64_t r) {
+  if (check_linear_shape(t, h, o, r) != QLORA_OK) return 0;
+  size_t b = lora_region_bytes(t, r);
+  if (t <= kGemvMaxTokens) b += gemv_region_bytes(t, o);
+  return b;
+}
+
+size_t qlora_bwd_workspace_bytes(int64_t t, int64_t h, int64_t o, int64_t r) {
+  if (check_linear_shape(t, h, o, r) != QLORA_OK) return 0;
+  return 2 * lora_region_bytes(t, r);
+}
+
+int qlora_profile_begin(int capacity) {
+  if (capacity < 1 || capacity > (1 << 20)) return QLORA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(prof::g.mu);
+  while (static_cast<int>(prof::g.events.size()) < 2 * capacity) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
+    prof::g.events.push_back(e);
+  }
+  if (static_cast<int>(prof::g.kinds.size()) < capacity) prof::g.kinds.resize(capacity);
+  prof::g.capacity = capacity;
+  prof::g.n = 0;
+  prof::g.overflow = false;
+  prof::g.on.store(true);
+  return QLORA_OK;
+}
+
+int qlora_profile_end(double* ms, int64_t* launches, int nkinds) {
+  std::lock_guard<std::mutex> lock(prof::g.mu);
+  prof::g.on.store(false);
+  if (ms) for (int k = 0; k < nkinds; ++k) ms[k] = 0.0;
+  if (launches) for (int k = 0; k < nkinds; ++k) launches[k] = 0;
+  for (int i = 0; i < prof::g.n; ++i) {
+    if (cudaEventSynchronize(prof::g.events[2 * i + 1]) != cudaSuccess) {
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, prof::g.events[2 * i], prof::g.events[2 * i + 1]) != cudaSuccess) {
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
+    const int k = prof::g.kinds[i];
+    if (k < nkinds) {
+      if (ms) ms[k] += t;
+      if (launches) launches[k] += 1;
+    }
+  }
+  if (prof::g.overflow) return QLORA_ERR_INVALID_ARG;
+  return prof::g.n;
+}
+
+const char* qlora_kernel_name(int kind) {
+  if (kind < 0 || kind >= prof::kKinds) return "unknown";
+  return prof::kNames[kind];
+}
+
+int qlora_get_last_status(qlora_stream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  return static_cast<int>(v);
+}
+
+int nf4_quantize(const float* Wt, const nf4_weight* q, qlora_stream_t stream) {
+  if (!Wt) return QLORA_ERR_INVALID_ARG;
+  int rc = check_weight(q);
+  if (rc) return rc;
+  if (!aligned16(Wt)) return QLORA_ERR_MISALIGNED;
+  int dev;
+  if ((rc = current_device(&dev))) return rc;
+  const int64_t nblocks = q->out_features * q->in_features / 64;
+  const int64_t ngroups = (nblocks + 255) / 256;
+  const int grid = static_cast<int>(std::min<int64_t>(ngroups, int64_t(sm_count(dev)) * 4));
+  {
+    prof::Scope ps(prof::kQuant, reinterpret_cast<cudaStream_t>(stream));
+    nf4_quantize_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        Wt, q->codes, q->absmax_q8, q->absmax_s2, nblocks, device_table());
+  }
+  return launch_status();
+}
+
+int nf4_dequantize(const nf4_weight* q, uint16_t* Wt_out, qlora_stream_t stream) {
+  if (!Wt_out) return QLORA_ERR_INVALID_ARG;
+  int rc = check_weight(q);
+  if (rc) return rc;
+  if (!aligned16(Wt_out)) return QLORA_ERR_MISALIGNED;
+  int dev;
+  if ((rc = current_device(&dev))) return rc;
+  const int64_t nitems = q->out_features * q->in_features / 8;
+  const int64_t want = (nitems + 4 * 256 - 1) / (4 * 256);
+  const int grid = static_cast<int>(std::min<int64_t>(want, int64_t(sm_count(dev)) * 8));
+  {
+    prof::Scope ps(prof::kDequant, reinterpret_cast<cudaStream_t>(stream));
+    nf4_dequantize_kernel<<<std::max(grid, 1), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        q->codes, q->absmax_q8, q->absmax_s2, Wt_out, nitems, device_table());
+  }
+  return launch_status();
+}
+
+int qlora_linear_fwd(const uint16_t* X, int64_t t, const nf4_weight* W, const uint16_t* L1,
+                     const uint16_t* L2, int64_t r, float s, uint16_t* Y, uint16_t* sT_out,
+                     void* workspace, size_t ws_bytes, qlora_stream_t stream) {
+  if (!X || !L1 || !L2 || !Y) return QLORA_ERR_INVALID_ARG;
+  if (!std::isfinite(s)) return QLORA_ERR_INVALID_ARG;
+  int rc = check_weight(W);
+  if (rc) return rc;
+  const int64_t h = W->in_features, o = W->out_features;
+  if ((rc = check_linear_shape(t, h, o, r))) return rc;
+  if (!aligned16(X) || !aligned16(L1) || !aligned16(L2) || !aligned16(Y) ||
+      (sT_out && !aligned16(sT_out)) || (workspace && !aligned16(workspace)))
+    return QLORA_ERR_MISALIGNED;
+  if (!workspace || ws_bytes < qlora_fwd_workspace_bytes(t, h, o, r)) return QLORA_ERR_WORKSPACE;
+  int dev;
+  if ((rc = current_device(&dev))) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int sms = sm_count(dev);
+  LoraWs ws = carve_lora(workspace, t, r);
+
+  // T = X . L1 (t x r), then sT = bf16(s . T)
+  CUtensorMap mX, mL1;
+  if (!map_bf16(&mX, X, h, t, 64, 128) || !map_bf16(&mL1, L1, r, h, 64, 64)) return QLORA_ERR_CUDA;
+
+  if (t <= kGemvMaxTokens) {
+    float* Y32 = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) +
+                                          lora_region_bytes(t, r));
+    if (cudaMemsetAsync(ws.acc32, 0, static_cast<size_t>(t) * r * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(Y32, 0, static_cast<size_t>(t) * o * 4, st) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    if ((rc = launch_tc_gemm<false, true>(mX, mL1, t, r, h, 1.0f, kOutAtomicRowMajor, ws.acc32, r,
+                                          sms, st)))
+      return rc;
+    GemvArgs ga{};
+    ga.codes = W->codes;
+    ga.q8 = W->absmax_q8;
+    ga.s2 = W->absmax_s2;
+    ga.X = X;
+    ga.Y32 = Y32;
+    ga.h = h;
+    ga.o = o;
+    ga.t = static_cast<int>(t);
+    ga.tab = device_table();
+    const int64_t nblk = h / 64;
+    const int64_t row_ctas = (o + 255) / 256;
+    // enough K slices for ~4 CTAs (16 warps) per SM
+    int64_t splits = std::max<int64_t>(1, (int64_t(sms) * 4 + row_ctas - 1) / row_ctas);
+    splits = std::min(splits, nblk);
+    ga.blocks_per_split = static_cast<int>((nblk + splits - 1) / splits);
+    const int64_t ysplits = (nblk + ga.blocks_per_split - 1) / ga.blocks_per_split;
+    dim3 grid(static_cast<unsigned>(row_ctas), static_cast<unsigned>(ysplits));
+    {
+      prof::Scope ps(prof::kGemv, st);
+      if (t <= 8)
+        nf4_gemv_kernel<1><<<grid, 128, 0, st>>>(ga);
+      else
+        nf4_gemv_kernel<2><<<grid, 128, 0, st>>>(ga);
+    }
+    if ((rc = launch_status())) return rc;
+    dim3 fgrid(static_cast<unsigned>((o + 255) / 256), static_cast<unsigned>(t));
+    {
+      prof::Scope ps(prof::kGemvFinalize, st);
+      gemv_lora_finalize_kernel<<<fgrid, 256, 0, st>>>(Y32, ws.acc32, L2, Y, o,
+                                                       static_cast<int>(r), s);
+    }
+    if ((rc = launch_status())) return rc;
+    if (sT_out) {
+      const int64_t count = t * r;
+      prof::Scope ps(prof::kScaleRound, st);
+      lora_scale_round_kernel<<<static_cast<unsigned>((count + 255) / 256), 256, 0, st>>>(
+          ws.acc32, sT_out, nullptr, count, s);
+      if ((rc = launch_status())) return rc;
+    }
+    return QLORA_OK;
+  }
+
+  uint16_t* sT = ws.b16;
+  if ((rc = lora_down<true>(mX, mL1, t, h, r, s, ws, sT, sT_out, sms, st))) return rc;
+
+  // Y = X . W' + sT . L2
+  CUtensorMap mA, mP, mA2, mB2;
+  if (!map_bf16(&mA, X, h, t, 64, 128) ||
+      !make_map_2d(&mP, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, h / 2, o, h / 2, 32, 256, false) ||
+      !map_bf16(&mA2, sT, r, t, 64, 128) || !map_bf16(&mB2, L2, o, r, 64, 64))
+    return QLORA_ERR_CUDA;
+  Nf4GemmArgs ga{};
+  ga.q8 = W->absmax_q8;
+  ga.s2 = W->absmax_s2;
+  ga.h = h;
+  ga.M = static_cast<int>(t);
+  ga.N = static_cast<int>(o);
+  ga.num_kb = static_cast<int>(h / 64);
+  ga.num_lkb = static_cast<int>((r + 63) / 64);
+  ga.out = Y;
+  ga.tab = device_table();
+  dim3 grid(static_cast<unsigned>((o + 255) / 256), static_cast<unsigned>((t + 127) / 128));
+  {
+    prof::Scope ps(prof::kGemmFwd, st);
+    nf4_gemm_kernel<false><<<grid, tc::kThreads, tc::nf4_gemm_smem_bytes(), st>>>(mA, mP, mA2,
+                                                                                mB2, ga);
+  }
+  return launch_status();
+}
+
+int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t t, const nf4_weight* W,
+                     const uint16_t* L1, const uint16_t* L2, int64_t r, float s,
+                     const uint16_t* sT_saved, uint16_t* dX, float* dL1, float* dL2,
+                     void* workspace, size_t ws_bytes, qlora_stream_t stream) {
+  if (!dY || !X || !L1 || !L2 || !dX || !dL1 || !dL2) return QLORA_ERR_INVALID_ARG;
+  if (!std::isfinite(s)) return QLORA_ERR_INVALID_ARG;
+  int rc = check_weight(W);
+  if (rc) return rc;
+  const int64_t h = W->in_features, o = W->out_features;
+  if ((rc = check_linear_shape(t, h, o, r))) return rc;
+  if (!aligned16(dY) || !aligned16(X) || !aligned16(L1) || !aligned16(L2) || !aligned16(dX) ||
+      !aligned16(dL1) || !aligned16(dL2) || (sT_saved && !aligned16(sT_saved)) ||
+      (workspace && !aligned16(workspace)))
+    return QLORA_ERR_MISALIGNED;
+  if (!workspace || ws_bytes < qlora_bwd_workspace_bytes(t, h, o, r)) return QLORA_ERR_WORKSPACE;
+  int dev;
+  if ((rc = current_device(&dev))) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int sms = sm_count(dev);
+  LoraWs wsU = carve_lora(workspace, t, r);
+  LoraWs wsT = carve_lora(reinterpret_cast<uint8_t*>(workspace) + lora_region_bytes(t, r), t, r);
+
+  // sU = bf16(s . dY . L2^T): A = dY (t x o, K-major), B[k=j][n=c] = L2[c][j] (K-major)
+  CUtensorMap mdY, mL2k;
+  if (!map_bf16(&mdY, dY, o, t, 64, 128) ||
+      !map_bf16(&mL2k, L2, o, r, 64, static_cast<uint32_t>((r + 15) / 16 * 16)))
+    return QLORA_ERR_CUDA;
+  uint16_t* sU = wsU.b16;
+  if ((rc = lora_down<false>(mdY, mL2k, t, o, r, s, wsU, sU, nullptr, sms, st))) return rc;
+
+  // sT = bf16(s . X . L1) unless the forward's copy was passed in
+  const uint16_t* sT = sT_saved;
+  if (!sT) {
+    CUtensorMap mX, mL1;
+    if (!map_bf16(&mX, X, h, t, 64, 128) || !map_bf16(&mL1, L1, r, h, 64, 64)) return QLORA_ERR_CUDA;
+    if ((rc = lora_down<true>(mX, mL1, t, h, r, s, wsT, wsT.b16, nullptr, sms, st))) return rc;
+    sT = wsT.b16;
+  }
+
+  // dX = dY . W'^T + sU . L1^T
+  {
+    CUtensorMap mA, mP, mA2, mB2;
+    if (!map_bf16(&mA, dY, o, t, 64, 128) ||
+        !make_map_2d(&mP, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, h / 2, o, h / 2, 32, 64, false) ||
+        !map_bf16(&mA2, sU, r, t, 64, 128) || !map_bf16(&mB2, L1, r, h, 64, 256))
+      return QLORA_ERR_CUDA;
+    Nf4GemmArgs ga{};
+    ga.q8 = W->absmax_q8;
+    ga.s2 = W->absmax_s2;
+    ga.h = h;
+    ga.M = static_cast<int>(t);
+    ga.N = static_cast<int>(h);
+    ga.num_kb = static_cast<int>(o / 64);
+    ga.num_lkb = static_cast<int>((r + 63) / 64);
+    ga.out = dX;
+    ga.tab = device_table();
+    dim3 grid(static_cast<unsigned>((h + 255) / 256), static_cast<unsigned>((t + 127) / 128));
+    {
+      prof::Scope ps(prof::kGemmBwd, st);
+      nf4_gemm_kernel<true><<<grid, tc::kThreads, tc::nf4_gemm_smem_bytes(), st>>>(mA, mP, mA2,
+                                                                                 mB2, ga);
+    }
+    if ((rc = launch_status())) return rc;
+  }
+
+  // dL1 = X^T . sU (h x r) and dL2^T = dY^T . sT (o x r), reductions over the t tokens
+  if (cudaMemsetAsync(dL1, 0, static_cast<size_t>(h) * r * 4, st) != cudaSuccess ||
+      cudaMemsetAsync(dL2, 0, static_cast<size_t>(r) * o * 4, st) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  CUtensorMap mXmn, msU, mdYmn, msT;
+  if (!map_bf16(&mXmn, X, h, t, 64, 64) || !map_bf16(&msU, sU, r, t, 64, 64) ||
+      !map_bf16(&mdYmn, dY, o, t, 64, 64) || !map_bf16(&msT, sT, r, t, 64, 64))
+    return QLORA_ERR_CUDA;
+  if ((rc = launch_tc_gemm<true, true>(mXmn, msU, h, r, t, 1.0f, kOutAtomicRowMajor, dL1, r, sms,
+                                       st)))
+    return rc;
+  return launch_tc_gemm<true, true>(mdYmn, msT, o, r, t, 1.0f, kOutAtomicTransposed, dL2, o, sms,
+                                    st);
+}
+
+}  // extern "C"

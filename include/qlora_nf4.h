@@ -1,0 +1,182 @@
+/*
+ * qlora_nf4.h -- C ABI of the QLoRA NF4 frozen-base linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The method (QLoRA, Dettmers et al., arXiv:2305.14314), as the source pages state it:
+ *   - a frozen base weight W (h x o) is stored as 4-bit NormalFloat codes in blocks of 64
+ *     weights, each block with an absmax scale ("QLoRA in LLMs", tensortonic.com, section 3
+ *     "How LoRA and Quantization Fit Together" and section 5 "NF4"; "QLoRA: Efficient
+ *     Finetuning of Quantized LLMs", mchromiak.github.io, "1. NormalFloat");
+ *   - the block scales are themselves quantized to 8 bits, with one higher-precision scale
+ *     per 256 of them ("2. Double quantization: Compress the scales too"; "A worked memory
+ *     budget for 65 billion weights"; "QLoRA in LLMs" section 6);
+ *   - for compute, blocks are dequantized on the fly to bf16 and contracted with the
+ *     activations ("QLoRA: the paper that put large-model fine-tuning on a desk",
+ *     goodomens.studio, "The core move"), and a trainable low-rank adapter is added:
+ *     Y = X.W + s.X.L1.L2 ("The algebra: How two small matrices change a layer"; s = alpha/r,
+ *     "QLoRA in LLMs" section 3);
+ *   - gradients reach the adapters through the frozen base, which receives none ("One
+ *     training step, from input to update"; "QLoRA in LLMs" section 4).
+ *
+ * Storage layout used throughout (the readings of the pages are stated in the design notes):
+ *   Wt      the weight stored transposed, o x h row-major ("out x in"); W' = Wt^T.
+ *   block   64 consecutive elements of Wt's flat row-major order (so h % 64 == 0).
+ *   codes   n/2 bytes; element 2j of the flat order is the high nibble of byte j.
+ *   q8      n/64 bytes: the 8-bit first-level scale of each block.
+ *   s2      ceil(n/16384) floats: one fp32 second-level scale per 256 blocks.
+ *   w'      bf16_rn( level[code] * (float(q8[b]) * s2[b/256]) ), two fp32 multiplies.
+ *   bf16    passed as uint16_t bit patterns.
+ *
+ * Conventions for every call:
+ *   - All pointers are DEVICE pointers owned by the caller, each aligned to 16 bytes, unless
+ *     a parameter says otherwise. The library never allocates, frees or synchronises device
+ *     memory except where stated (qlora_get_last_status synchronises its stream).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default stream).
+ *   - Outputs are overwritten, never accumulated into. Inputs are not modified.
+ *   - Return value: 0 on success; a negative QLORA_ERR_* code when the host-side checks
+ *     reject the arguments or a launch fails, in which case nothing was launched (for
+ *     argument errors) or the launch error is returned. Faults the kernels detect while
+ *     running (non-finite weights, an internal wait that timed out) are OR-ed into a device
+ *     status word, read and cleared by qlora_get_last_status.
+ *   - The device must be an sm_100 GPU (B200); any other device gives
+ *     QLORA_ERR_UNSUPPORTED_DEVICE.
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QLORA_API __attribute__((visibility("default")))
+#else
+#define QLORA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream handle, layout-compatible with cudaStream_t. */
+typedef struct CUstream_st *qlora_stream_t;
+
+/* Host-side status codes (negative) returned by every call. */
+enum {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID_ARG = -1,       /* null pointer, bad rank r, t < 1, bad scalar           */
+  QLORA_ERR_BAD_SHAPE = -2,         /* h % 64 != 0, o % 64 != 0, size overflow               */
+  QLORA_ERR_MISALIGNED = -3,        /* a pointer is not 16-byte aligned                      */
+  QLORA_ERR_WORKSPACE = -4,         /* workspace pointer NULL or smaller than required       */
+  QLORA_ERR_CUDA = -5,              /* a CUDA runtime call or kernel launch failed           */
+  QLORA_ERR_UNSUPPORTED_DEVICE = -6 /* the current device is not sm_100                      */
+};
+
+/* Device-side fault bits (positive), OR-ed into the status word by the kernels. */
+enum {
+  QLORA_DEV_NONFINITE = 1,          /* nf4_quantize met a NaN or infinite weight             */
+  QLORA_DEV_TIMEOUT = 2             /* a kernel's bounded internal wait expired; outputs of
+                                       that call are unspecified                              */
+};
+
+/* A packed NF4 weight: caller-owned device buffers plus the logical shape.
+ * Block size 64 and scale-group size 256 are fixed by the method. */
+typedef struct nf4_weight {
+  uint8_t *codes;        /* n/2 bytes, n = out_features * in_features                        */
+  uint8_t *absmax_q8;    /* n/64 bytes                                                        */
+  float *absmax_s2;      /* ceil(n/16384) floats                                             */
+  int64_t out_features;  /* o: rows of Wt                                                     */
+  int64_t in_features;   /* h: columns of Wt, h % 64 == 0                                     */
+} nf4_weight;
+
+/* The 16 NF4 levels (ascending fp32, exact zero at index 7, ends -1 and +1), as this library
+ * derives them from standard-normal quantiles ("QLoRA in LLMs" section 5; "Idea one: NF4" on
+ * goodomens.studio). Host call, no device needed. levels: host array of 16 floats;
+ * midpoints: host array of 15 floats (decision thresholds) or NULL. Returns 0 or
+ * QLORA_ERR_INVALID_ARG when levels is NULL. */
+QLORA_API int qlora_nf4_codebook(float *levels, float *midpoints);
+
+/* nf4_quantize -- blockwise NF4 quantization with double-quantized scales.
+ * Follows "QLoRA in LLMs" section 2 (absmax scale, normalise, round to the nearest
+ * representable value), section 5 (NF4 levels) and section 6 (double quantization), and
+ * "2. Double quantization" on mchromiak.github.io.
+ *   Wt  device, fp32, o x h row-major (o = q->out_features, h = q->in_features), read only.
+ *   q   host pointer to a descriptor whose device buffers receive codes, q8 and s2.
+ * Per block: c1 = max|w|; x = w / c1 (fp32, round to nearest); code = number of midpoints
+ * strictly below x (a block with c1 == 0 takes code 7). Per group of 256 blocks (the last may
+ * be shorter): s2 = max(c1) / 255; q8 = clamp(round_half_even(c1 / s2), 0, 255) (0 when s2
+ * is 0). The codes use the exact c1, not the 8-bit scale. A non-finite weight sets
+ * QLORA_DEV_NONFINITE; the outputs for its group are then unspecified.
+ * Errors: INVALID_ARG (NULL), BAD_SHAPE (h % 64 != 0, o < 1), MISALIGNED. */
+QLORA_API int nf4_quantize(const float *Wt, const nf4_weight *q, qlora_stream_t stream);
+
+/* nf4_dequantize -- reconstruct the bf16 weight Wt' (o x h row-major) from a packed weight.
+ * "QLoRA in LLMs" section 3 (dequantized into BF16 for a calculation); "1. NormalFloat" on
+ * mchromiak.github.io. Wt_out: device, bf16 bits, o*h elements. Bit-exact definition:
+ * w' = bf16_rn(level[code] * (float(q8) * s2)). Errors: INVALID_ARG, BAD_SHAPE, MISALIGNED. */
+QLORA_API int nf4_dequantize(const nf4_weight *q, uint16_t *Wt_out, qlora_stream_t stream);
+
+/* qlora_linear_fwd -- Y = X.W' + s.X.L1.L2 for one adapted linear layer.
+ * "The algebra" (mchromiak.github.io): X is t x h, W is h x o, L1 is h x r, L2 is r x o,
+ * scalar s; "QLoRA in LLMs" section 3-4; the base block is dequantized on the fly and
+ * discarded ("The core move" on goodomens.studio).
+ *   X        device bf16, t x h row-major.          t >= 1.
+ *   W        host pointer to the packed weight (o x h stored); h % 64 == 0, o % 64 == 0.
+ *   L1       device bf16, h x r row-major.          16 <= r <= 256, r % 16 == 0.
+ *   L2       device bf16, r x o row-major.
+ *   s        the adapter scale (alpha / r); any finite value.
+ *   Y        device bf16, t x o row-major (output).
+ *   sT_out   device bf16, t x r (output, bf16(s . X.L1), kept for the backward) or NULL.
+ *   workspace, ws_bytes: device scratch of at least qlora_fwd_workspace_bytes(t, h, o, r)
+ *            bytes, caller-owned; contents on entry are ignored.
+ * Compute: bf16 operands, fp32 accumulation; the LoRA term uses the bf16-rounded
+ * sT = bf16(s . X.L1), folded into the same accumulator as X.W'. */
+QLORA_API int qlora_linear_fwd(const uint16_t *X, int64_t t, const nf4_weight *W,
+                     const uint16_t *L1, const uint16_t *L2, int64_t r, float s,
+                     uint16_t *Y, uint16_t *sT_out,
+                     void *workspace, size_t ws_bytes, qlora_stream_t stream);
+
+/* qlora_linear_bwd -- gradients of the adapted linear; the frozen W gets none.
+ * "One training step, from input to update" (mchromiak.github.io); "QLoRA in LLMs" section 4.
+ *   dY       device bf16, t x o (upstream gradient).     X: device bf16, t x h.
+ *   W, L1, L2, r, s: as in qlora_linear_fwd.
+ *   sT_saved device bf16, t x r = bf16(s . X.L1) from the forward, or NULL to recompute it.
+ *   dX       device bf16, t x h (output) = dY.W'^T + sU.L1^T with sU = bf16(s . dY.L2^T).
+ *   dL1      device fp32, h x r (output) = X^T . sU.
+ *   dL2      device fp32, r x o (output) = sT^T . dY.
+ *   workspace, ws_bytes: at least qlora_bwd_workspace_bytes(t, h, o, r) bytes. */
+QLORA_API int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, int64_t t, const nf4_weight *W,
+                     const uint16_t *L1, const uint16_t *L2, int64_t r, float s,
+                     const uint16_t *sT_saved, uint16_t *dX, float *dL1, float *dL2,
+                     void *workspace, size_t ws_bytes, qlora_stream_t stream);
+
+/* Workspace sizes in bytes for the two linear calls (host functions, no device needed).
+ * Return 0 for shapes the calls would reject. */
+QLORA_API size_t qlora_fwd_workspace_bytes(int64_t t, int64_t h, int64_t o, int64_t r);
+QLORA_API size_t qlora_bwd_workspace_bytes(int64_t t, int64_t h, int64_t o, int64_t r);
+
+/* Synchronise `stream`, then return and clear the device status word of the current device:
+ * 0, or an OR of QLORA_DEV_* bits, or QLORA_ERR_CUDA if the synchronisation failed. */
+QLORA_API int qlora_get_last_status(qlora_stream_t stream);
+
+/* Kernel timing (measurement support, not part of the method). While a profile is open on
+ * the current device, the library records a pair of CUDA events around each of its kernel
+ * launches, on the launching stream. qlora_profile_begin(capacity) opens a profile for up to
+ * `capacity` launches (events are created once and reused; no device memory is allocated).
+ * qlora_profile_end synchronises the last recorded event, closes the profile and writes, for
+ * each kernel kind k < nkinds, the summed device time in milliseconds (ms[k]) and the number
+ * of launches (launches[k]); it returns the number of launches recorded, or QLORA_ERR_CUDA,
+ * or QLORA_ERR_INVALID_ARG if the profile overflowed its capacity. Kinds are numbered
+ * 0 .. QLORA_KERNEL_KINDS-1 and named by qlora_kernel_name. Not thread-safe across
+ * concurrent calls into the library while open. */
+#define QLORA_KERNEL_KINDS 8
+QLORA_API int qlora_profile_begin(int capacity);
+QLORA_API int qlora_profile_end(double *ms, int64_t *launches, int nkinds);
+QLORA_API const char *qlora_kernel_name(int kind);
+
+/* A static, human-readable name for any QLORA_* code (never NULL). */
+QLORA_API const char *qlora_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_NF4_H */

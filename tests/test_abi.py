@@ -1,0 +1,111 @@
+"""The C-ABI library loads without a GPU, exports every function include/qlora_nf4.h declares,
+derives the same NF4 codebook as the oracle, and rejects bad arguments on the host before
+touching CUDA (these calls never launch anything)."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from bit_quantized_lora_03_b200 import binding as B
+from bit_quantized_lora_03_b200 import build as build_mod
+from oracle import nf4_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qlora_nf4.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return B.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"QLORA_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)))
+
+
+def test_header_declares_the_four_calls_and_helpers():
+    names = declared_functions()
+    for required in ["nf4_quantize", "nf4_dequantize", "qlora_linear_fwd", "qlora_linear_bwd",
+                     "qlora_get_last_status", "qlora_status_string"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert names
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(names) <= set(B.SIGNATURES), "binding signatures must cover the header"
+
+
+def test_library_links_no_gpu_driver():
+    out = os.popen(f"ldd {build_mod.LIB_PATH}").read()
+    assert "libcuda.so" not in out and "libcudart.so" not in out
+
+
+def test_codebook_matches_oracle_bit_exactly(lib):
+    lv, md = B.codebook()
+    assert np.array_equal(np.array(lv, np.float32), O.nf4_codebook())
+    assert np.array_equal(np.array(md, np.float32), O.nf4_midpoints())
+    assert lib.qlora_nf4_codebook(None, None) == B.QLORA_ERR_INVALID_ARG
+
+
+def test_status_strings(lib):
+    for code in [0, -1, -2, -3, -4, -5, -6, 1, 2, 3, 12345]:
+        s = B.status_string(code)
+        assert isinstance(s, str) and s
+
+
+def test_workspace_sizes(lib):
+    assert lib.qlora_fwd_workspace_bytes(4096, 4096, 4096, 64) >= 4096 * 64 * 6
+    assert lib.qlora_bwd_workspace_bytes(4096, 4096, 4096, 64) >= 2 * 4096 * 64 * 6
+    # the decode path also keeps a t x o fp32 accumulator
+    assert lib.qlora_fwd_workspace_bytes(16, 4096, 11008, 16) >= 16 * 11008 * 4
+    assert lib.qlora_fwd_workspace_bytes(0, 4096, 4096, 64) == 0
+    assert lib.qlora_fwd_workspace_bytes(8, 100, 4096, 64) == 0      # h % 64 != 0
+    assert lib.qlora_fwd_workspace_bytes(8, 4096, 4096, 24) == 0     # r % 16 != 0
+    assert lib.qlora_bwd_workspace_bytes(8, 4096, 4096, 512) == 0    # r > 256
+
+
+def _desc(codes=0x1000, q8=0x2000, s2=0x3000, o=128, h=128):
+    return B.NF4WeightDesc(codes, q8, s2, o, h)
+
+
+def test_host_validation_rejects_before_launch(lib):
+    d = _desc()
+    assert lib.nf4_quantize(None, ctypes.byref(d), None) == B.QLORA_ERR_INVALID_ARG
+    assert lib.nf4_quantize(0x1000, None, None) == B.QLORA_ERR_INVALID_ARG
+    bad_h = _desc(h=100)
+    assert lib.nf4_quantize(0x1000, ctypes.byref(bad_h), None) == B.QLORA_ERR_BAD_SHAPE
+    zero_o = _desc(o=0)
+    assert lib.nf4_quantize(0x1000, ctypes.byref(zero_o), None) == B.QLORA_ERR_BAD_SHAPE
+    mis = _desc(codes=0x1001)
+    assert lib.nf4_quantize(0x1000, ctypes.byref(mis), None) == B.QLORA_ERR_MISALIGNED
+    assert lib.nf4_quantize(0x1004, ctypes.byref(d), None) == B.QLORA_ERR_MISALIGNED
+    null_codes = _desc(codes=0)
+    assert lib.nf4_dequantize(ctypes.byref(null_codes), 0x1000, None) == B.QLORA_ERR_INVALID_ARG
+    assert lib.nf4_dequantize(ctypes.byref(d), None, None) == B.QLORA_ERR_INVALID_ARG
+    assert lib.nf4_dequantize(ctypes.byref(d), 0x1008, None) == B.QLORA_ERR_MISALIGNED
+
+    P = 0x10000
+    fwd = lib.qlora_linear_fwd
+    assert fwd(None, 4, ctypes.byref(d), P, P, 16, 1.0, P, None, P, 1 << 30, None) == B.QLORA_ERR_INVALID_ARG
+    assert fwd(P, 0, ctypes.byref(d), P, P, 16, 1.0, P, None, P, 1 << 30, None) == B.QLORA_ERR_INVALID_ARG
+    assert fwd(P, 4, ctypes.byref(d), P, P, 24, 1.0, P, None, P, 1 << 30, None) == B.QLORA_ERR_INVALID_ARG
+    assert fwd(P, 4, ctypes.byref(d), P, P, 16, float("nan"), P, None, P, 1 << 30, None) == B.QLORA_ERR_INVALID_ARG
+    d_o = _desc(o=100)
+    assert fwd(P, 4, ctypes.byref(d_o), P, P, 16, 1.0, P, None, P, 1 << 30, None) == B.QLORA_ERR_BAD_SHAPE
+    assert fwd(P + 2, 4, ctypes.byref(d), P, P, 16, 1.0, P, None, P, 1 << 30, None) == B.QLORA_ERR_MISALIGNED
+    assert fwd(P, 4, ctypes.byref(d), P, P, 16, 1.0, P, None, None, 0, None) == B.QLORA_ERR_WORKSPACE
+    assert fwd(P, 4, ctypes.byref(d), P, P, 16, 1.0, P, None, P, 16, None) == B.QLORA_ERR_WORKSPACE
+
+    bwd = lib.qlora_linear_bwd
+    assert bwd(P, P, 4, ctypes.byref(d), P, P, 16, 1.0, None, P, P, None, P, 1 << 30, None) == B.QLORA_ERR_INVALID_ARG
+    assert bwd(P, P, 4, ctypes.byref(d), P, P, 16, 1.0, None, P, P, P + 4, P, 1 << 30, None) == B.QLORA_ERR_MISALIGNED
+    assert bwd(P, P, 4, ctypes.byref(d), P, P, 16, 1.0, None, P, P, P, P, 8, None) == B.QLORA_ERR_WORKSPACE

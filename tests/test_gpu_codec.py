@@ -1,0 +1,87 @@
+"""GPU parity of nf4_quantize / nf4_dequantize against the CPU oracle, bit for bit.
+
+Inputs: the seeded workloads (single 1024 x 1024 linear; every linear of a LLaMA-7B-shaped
+layer with 1% outliers at +-8 sigma; the decode-shape weights), ragged shapes (partial last
+scale group, one block, odd row counts), and the degenerate cases (all-zero blocks and groups,
+exactly representable blocks, non-finite weights -> status bit)."""
+
+import numpy as np
+import pytest
+import torch
+
+from bit_quantized_lora_03_b200 import binding as B
+from bit_quantized_lora_03_b200 import inputs
+from oracle import nf4_oracle as O
+
+from gpu_util import oracle_packed_rows, require_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def _check_full(Wt: torch.Tensor):
+    p = B.nf4_quantize(Wt.cuda())
+    deq = B.nf4_dequantize(p)
+    assert B.last_status() == 0
+    ref = O.nf4_quantize(Wt.numpy())
+    assert np.array_equal(p.codes.cpu().numpy(), ref.codes), "packed codes differ"
+    assert np.array_equal(p.absmax_q8.cpu().numpy(), ref.absmax_q8), "8-bit scales differ"
+    assert np.array_equal(p.absmax_s2.cpu().numpy().view(np.uint32),
+                          ref.absmax_s2.view(np.uint32)), "second-level scales differ"
+    got = deq.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got, O.nf4_dequantize_bits(ref)), "dequantized bf16 differs"
+
+
+def test_single_linear_1024():
+    _check_full(inputs.single_linear_1024().Wt)
+
+
+@pytest.mark.parametrize("o,h", [(1, 64), (3, 128), (5, 64 * 300), (257, 192), (64, 4096 + 64)])
+def test_ragged_shapes(o, h):
+    g = torch.Generator().manual_seed(o * 1000 + h)
+    _check_full(torch.randn(o, h, generator=g) * 0.02)
+
+
+@pytest.mark.parametrize("i", range(7))
+def test_llama7b_layer_with_outliers(i):
+    name, h, o = inputs.LLAMA7B_LINEARS[i]
+    _check_full(inputs.weight_f32(o, h, 200 + i, outliers=True))
+
+
+def test_decode_weight_4096x11008():
+    _check_full(inputs.decode_gemv_weights()[0][1])
+
+
+def test_degenerate_blocks():
+    q = O.nf4_codebook()
+    W = torch.zeros(4, 64 * 130)
+    W[1, :64] = torch.from_numpy(q[np.arange(64) % 16] * np.float32(0.5))   # representable
+    W[2, 64:128] = 1e-30                                                    # tiny block
+    W[3, -64:] = -3.0                                                       # one-signed block
+    _check_full(W)
+    _check_full(torch.zeros(2, 64 * 300))
+
+
+def test_nonfinite_sets_status_bit():
+    W = torch.randn(8, 256) * 0.02
+    W[3, 17] = float("nan")
+    B.last_status()
+    B.nf4_quantize(W.cuda())
+    assert B.last_status() & B.QLORA_DEV_NONFINITE
+    assert B.last_status() == 0          # reading clears it
+
+
+def test_sampled_rows_of_the_largest_decode_weight():
+    """8192 x 28672 packed on the GPU; 24 rows recomputed by the oracle one by one."""
+    Wt = inputs.decode_gemv_weights()[1][1]
+    p = B.nf4_quantize(Wt.cuda())
+    deq = B.nf4_dequantize(p)
+    rows = sorted(set(torch.randint(0, Wt.shape[0], (24,), generator=torch.Generator().manual_seed(5)).tolist()
+                      + [0, Wt.shape[0] - 1]))
+    ref = oracle_packed_rows(Wt.numpy(), rows)
+    got = deq[rows].float().cpu().numpy()
+    assert np.array_equal(got.view(np.uint32), ref.astype(np.float32).view(np.uint32))
