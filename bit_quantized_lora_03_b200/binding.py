@@ -23,6 +23,8 @@ QLORA_ERR_MISALIGNED = -3
 QLORA_ERR_WORKSPACE = -4
 QLORA_ERR_CUDA = -5
 QLORA_ERR_UNSUPPORTED_DEVICE = -6
+QLORA_ERR_SCRATCH_LIMIT = -7
+QLORA_STATIC_SCRATCH_BYTES = 8 << 20
 QLORA_DEV_NONFINITE = 1
 QLORA_DEV_TIMEOUT = 2
 
@@ -44,6 +46,8 @@ SIGNATURES = {
     "qlora_profile_begin": (ctypes.c_int, [ctypes.c_int]),
     "qlora_profile_end": (ctypes.c_int, [_PTR, _PTR, ctypes.c_int]),
     "qlora_kernel_name": (ctypes.c_char_p, [ctypes.c_int]),
+    "qlora_linear_fwd_noalloc": (ctypes.c_int, [_PTR, _I64, _PTR, _PTR, _PTR, _I64,
+                                                ctypes.c_float, _PTR, _PTR, _PTR]),
 }
 KERNEL_KINDS = 8
 

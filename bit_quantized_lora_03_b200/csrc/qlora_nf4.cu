@@ -370,6 +370,8 @@ const char* qlora_status_string(int status) {
     case QLORA_ERR_WORKSPACE: return "QLORA_ERR_WORKSPACE: workspace missing or too small";
     case QLORA_ERR_CUDA: return "QLORA_ERR_CUDA: CUDA runtime or launch error";
     case QLORA_ERR_UNSUPPORTED_DEVICE: return "QLORA_ERR_UNSUPPORTED_DEVICE: not an sm_100 GPU";
+    case QLORA_ERR_SCRATCH_LIMIT:
+      return "QLORA_ERR_SCRATCH_LIMIT: shape needs more than the static scratch holds";
     case QLORA_DEV_NONFINITE: return "QLORA_DEV_NONFINITE: non-finite weight";
     case QLORA_DEV_TIMEOUT: return "QLORA_DEV_TIMEOUT: a kernel wait timed out";
     case QLORA_DEV_NONFINITE | QLORA_DEV_TIMEOUT:
@@ -678,3 +680,60 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t t, const nf4
 }
 
 }  // extern "C"
+
+// ==========================================================================================
+// Allocation-free forward: the caller's workspace replaced by a scratch array in the library's
+// own device image. The forward itself is qlora_linear_fwd, unchanged.
+// ==========================================================================================
+namespace {
+
+// One copy per device that loads the library, alive until the process exits.
+static __device__ __align__(256) unsigned char g_static_scratch[QLORA_STATIC_SCRATCH_BYTES];
+
+struct StaticScratch {
+  std::once_flag once;
+  void* ptr = nullptr;  // device address of g_static_scratch on this device
+  int rc = QLORA_ERR_CUDA;
+};
+StaticScratch g_scratch[kMaxDevices];
+
+// In host code the name g_static_scratch is only a host-side stand-in, not a device address:
+// the address a kernel may use is looked up once per device, with that device current.
+int static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return QLORA_ERR_UNSUPPORTED_DEVICE;
+  StaticScratch& sc = g_scratch[dev];
+  std::call_once(sc.once, [&] {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      sc.rc = QLORA_ERR_CUDA;
+      return;
+    }
+    sc.ptr = p;
+    sc.rc = QLORA_OK;
+  });
+  *out = sc.ptr;
+  return sc.rc;
+}
+
+}  // namespace
+
+extern "C" int qlora_linear_fwd_noalloc(const uint16_t* X, int64_t t, const nf4_weight* W,
+                                        const uint16_t* L1, const uint16_t* L2, int64_t r, float s,
+                                        uint16_t* Y, uint16_t* sT_out, qlora_stream_t stream) {
+  if (!W) return QLORA_ERR_INVALID_ARG;
+  const size_t need = qlora_fwd_workspace_bytes(t, W->in_features, W->out_features, r);
+  if (need > QLORA_STATIC_SCRATCH_BYTES) return QLORA_ERR_SCRATCH_LIMIT;
+  void* scratch = nullptr;
+  if (need != 0) {  // need == 0: invalid shape, let the forward's own checks report it
+    const int rc = static_scratch(&scratch);
+    if (rc != QLORA_OK) return rc;
+  }
+  return qlora_linear_fwd(X, t, W, L1, L2, r, s, Y, sT_out, scratch,
+                          scratch ? static_cast<size_t>(QLORA_STATIC_SCRATCH_BYTES) : 0, stream);
+}

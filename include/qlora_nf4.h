@@ -67,7 +67,9 @@ enum {
   QLORA_ERR_MISALIGNED = -3,        /* a pointer is not 16-byte aligned                      */
   QLORA_ERR_WORKSPACE = -4,         /* workspace pointer NULL or smaller than required       */
   QLORA_ERR_CUDA = -5,              /* a CUDA runtime call or kernel launch failed           */
-  QLORA_ERR_UNSUPPORTED_DEVICE = -6 /* the current device is not sm_100                      */
+  QLORA_ERR_UNSUPPORTED_DEVICE = -6, /* the current device is not sm_100                     */
+  QLORA_ERR_SCRATCH_LIMIT = -7      /* qlora_linear_fwd_noalloc: the shape needs more scratch
+                                       than QLORA_STATIC_SCRATCH_BYTES                        */
 };
 
 /* Device-side fault bits (positive), OR-ed into the status word by the kernels. */
@@ -147,6 +149,28 @@ QLORA_API int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, int64_t t,
                      const uint16_t *L1, const uint16_t *L2, int64_t r, float s,
                      const uint16_t *sT_saved, uint16_t *dX, float *dL1, float *dL2,
                      void *workspace, size_t ws_bytes, qlora_stream_t stream);
+
+/* qlora_linear_fwd_noalloc -- the same forward as qlora_linear_fwd, for callers that cannot
+ * allocate device memory. There is no counterpart in the QLoRA method: this is a deployment
+ * convenience. Some callers are handed only their input and output buffers (a plugin slot in
+ * a host framework, a serving loop whose memory budget is fixed at start-up) and have no way
+ * to obtain a workspace, and cudaMalloc/cudaFree may synchronise the whole device, which a
+ * latency-bound caller cannot afford.
+ * Instead of a caller workspace this call uses a scratch array of QLORA_STATIC_SCRATCH_BYTES
+ * that lives in the library's device image: every GPU that loads the library holds it until
+ * the process exits. The call allocates nothing and calls no allocating routine.
+ *   - Arguments and results: exactly those of qlora_linear_fwd without workspace/ws_bytes.
+ *   - Limit: shapes with qlora_fwd_workspace_bytes(t, h, o, r) > QLORA_STATIC_SCRATCH_BYTES
+ *     are rejected with QLORA_ERR_SCRATCH_LIMIT before anything is launched.
+ *   - The first call on a device looks up the array's device address (once per device, with
+ *     that device current); make that first call before any stream capture begins.
+ *   - All calls share the one array, and it keeps whatever the previous call left there (the
+ *     call clears the parts that must start at zero itself). Two calls whose kernels overlap on
+ *     the GPU, for example on two streams, race on the array: serialise them. */
+#define QLORA_STATIC_SCRATCH_BYTES (8u << 20)
+QLORA_API int qlora_linear_fwd_noalloc(const uint16_t *X, int64_t t, const nf4_weight *W,
+                                       const uint16_t *L1, const uint16_t *L2, int64_t r, float s,
+                                       uint16_t *Y, uint16_t *sT_out, qlora_stream_t stream);
 
 /* Workspace sizes in bytes for the two linear calls (host functions, no device needed).
  * Return 0 for shapes the calls would reject. */
