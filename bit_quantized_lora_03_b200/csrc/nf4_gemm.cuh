@@ -9,10 +9,11 @@
 //    A (X or dY) and the packed codes arrive by TMA; 8 producer warps turn each 64-weight
 //    block into bf16 (w' = bf16(level * (q8 * s2)), the exact nf4_dequantize values) and
 //    write it straight into the 128-byte-swizzled operand layout the MMA reads: K-major for
-//    the forward (rows of Wt are N), MN-major for the backward (rows of Wt are K). One thread
-//    issues tcgen05.mma into a 128 x 256 fp32 accumulator in tensor memory; the r/64 LoRA
-//    K-steps (A = sT or sU, B = L2 or L1, both by TMA) run first, then the h/64 (or o/64)
-//    weight K-steps. Four epilogue warps read TMEM and write bf16.
+//    the forward (rows of Wt are N), MN-major for the backward (rows of Wt are K). A CTA owns
+//    256 tokens x 256 columns: one thread issues tcgen05.mma into two 128 x 256 fp32
+//    accumulators in tensor memory (all 512 columns), so every dequantized weight tile feeds
+//    256 tokens. The r/64 LoRA K-steps (A = sT or sU, B = L2 or L1, both by TMA) run first,
+//    then the h/64 (or o/64) weight K-steps. The same 8 warps then drain TMEM to bf16.
 //
 // 2) tc_gemm_kernel<A_MN, B_MN>: a plain TMA-fed tcgen05 GEMM (both operands by TMA, either
 //    major-ness) with split-K and fp32 atomic or bf16 output, for the rank-r products
@@ -27,19 +28,19 @@
 namespace qlora {
 namespace tc {
 
-constexpr int BM = 128;        // tokens per tile (TMEM lanes)
-constexpr int BN = 256;        // output columns per tile (TMEM fp32 columns)
+constexpr int BM = 256;        // tokens per tile: two 128-lane TMEM accumulators
+constexpr int BN = 256;        // output columns per tile (fp32 TMEM columns per accumulator)
 constexpr int BK = 64;         // K per stage: one 128-byte swizzle row of bf16, one NF4 block
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;       // 16 KB
+constexpr int STAGES = 3;
+constexpr int A_HALF = 128 * BK * 2;       // 16 KB: one 128-token half of the A tile
+constexpr int A_BYTES = BM * BK * 2;       // 32 KB
 constexpr int B_BYTES = BN * BK * 2;       // 32 KB
 constexpr int P_BYTES = BN * BK / 2;       // 8 KB of packed codes
-constexpr int kEpiWarps = 4;               // warps 0-3: epilogue (TMEM lanes 0-127)
-constexpr int kDeqWarps = 8;               // warps 4-11: dequant producers
-constexpr int kTmaWarp = 12;
-constexpr int kMmaWarp = 13;
-constexpr int kThreads = 14 * 32;
-constexpr int kTmemCols = 256;
+constexpr int kWorkWarps = 8;              // warps 0-7: dequant producers, then epilogue
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 10 * 32;
+constexpr int kTmemCols = 512;
 
 constexpr size_t nf4_gemm_smem_bytes() {
   return 1024 /* alignment slack */ + STAGES * (A_BYTES + B_BYTES + P_BYTES) + 256;
@@ -71,6 +72,36 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// bf16x2 of (a * k, b * k): one packed fp32x2 multiply (IEEE round to nearest per lane, the
+// same two products as two separate multiplies), then round-to-nearest-even to bf16.
+__device__ __forceinline__ uint32_t scale_pack_bf16x2(float a, float b, uint64_t kk) {
+  uint64_t ab, r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(ab) : "f"(a), "f"(b));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(ab), "l"(kk));
+  float ra, rb;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(ra), "=f"(rb) : "l"(r));
+  return pack_bf16x2(ra, rb);
+}
+
+// Eight packed codes (one 32-bit word, element 2j in the high nibble of byte j) -> eight bf16
+// weights level[code] * k. The level table is 16 fp32 in shared memory; the byte offsets
+// 4*code of all eight nibbles come from two mask operations and one byte-permute each.
+__device__ __forceinline__ uint4 dequant8(uint32_t x, uint64_t kk, const float* lv) {
+  const uint32_t hi4 = (x >> 2) & 0x3C3C3C3Cu;   // byte j: 4 * high nibble
+  const uint32_t lo4 = (x << 2) & 0x3C3C3C3Cu;   // byte j: 4 * low nibble
+  const char* base = reinterpret_cast<const char*>(lv);
+  uint32_t w[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t oh = __byte_perm(hi4, 0u, 0x4440u + j);
+    const uint32_t ol = __byte_perm(lo4, 0u, 0x4440u + j);
+    const float a = *reinterpret_cast<const float*>(base + oh);
+    const float b = *reinterpret_cast<const float*>(base + ol);
+    w[j] = scale_pack_bf16x2(a, b, kk);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 template <bool kBwd>
 __global__ void __launch_bounds__(tc::kThreads, 1)
     nf4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmP,
@@ -78,6 +109,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                     const __grid_constant__ CUtensorMap tmB2, const Nf4GemmArgs args) {
   using namespace tc;
   extern __shared__ uint8_t smem_raw[];
+  __shared__ float lv[16];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
@@ -89,7 +121,6 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   uint64_t* acc_full = empty + STAGES;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
   volatile uint32_t* abort_flag = tmem_holder + 1;
-  float* lv = reinterpret_cast<float*>(tmem_holder + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * BN;
@@ -99,7 +130,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_ap[s], 1);
-      mbar_init(&full_b[s], kDeqWarps * 32);
+      mbar_init(&full_b[s], kWorkWarps * 32);
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
@@ -133,6 +164,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         if (i < args.num_lkb) {
           mbar_arrive_expect_tx(&full_ap[slot], A_BYTES + B_BYTES);
           tma_load_2d(a_dst, &tmA2, &full_ap[slot], i * BK, m0);
+          tma_load_2d(a_dst + A_HALF, &tmA2, &full_ap[slot], i * BK, m0 + 128);
           if (!kBwd) {
             // L2 (r x o), MN-major B: four 64-column atoms, 8 KB apart
 #pragma unroll
@@ -147,6 +179,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
           const int kb = i - args.num_lkb;
           mbar_arrive_expect_tx(&full_ap[slot], A_BYTES + P_BYTES);
           tma_load_2d(a_dst, &tmA, &full_ap[slot], kb * BK, m0);
+          tma_load_2d(a_dst + A_HALF, &tmA, &full_ap[slot], kb * BK, m0 + 128);
           if (!kBwd) {
             tma_load_2d(sP + slot * P_BYTES, &tmP, &full_ap[slot], kb * (BK / 2), n0);
           } else {
@@ -166,8 +199,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
-      constexpr uint32_t kIdescMain = idesc_bf16(BM, BN, false, kBwd);
-      constexpr uint32_t kIdescLora = idesc_bf16(BM, BN, false, !kBwd);
+      constexpr uint32_t kIdescMain = idesc_bf16(128, BN, false, kBwd);
+      constexpr uint32_t kIdescLora = idesc_bf16(128, BN, false, !kBwd);
       bool any = false;
       for (int i = 0; i < total; ++i) {
         const int slot = i % STAGES;
@@ -182,10 +215,13 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         const uint32_t b_addr = smem_addr(sB + slot * B_BYTES);
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t ad = sw128_desc(a_addr + kk * 32, 16, 1024);
           const uint64_t bd = b_mn ? sw128_desc(b_addr + kk * 2048, 8192, 1024)
                                    : sw128_desc(b_addr + kk * 32, 16, 1024);
-          umma_bf16(tmem_base, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const uint64_t ad = sw128_desc(a_addr + half * A_HALF + kk * 32, 16, 1024);
+            umma_bf16(tmem_base + half * BN, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         umma_commit(&empty[slot]);
         any = true;
@@ -194,70 +230,88 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       umma_commit(acc_full);
       if (*abort_flag && any) mbar_drain(acc_full, 0);
     }
-  } else if (warp >= kEpiWarps && warp < kEpiWarps + kDeqWarps) {
-    // ---------------- dequant producers: one 64-weight block per thread per stage ----------
-    const int p = threadIdx.x - kEpiWarps * 32;  // 0..255
+  } else {
+    // ---------------- warps 0-7: dequant producers (one 64-weight block per thread per
+    // stage), then the epilogue ---------------------------------------------------------
+    const int p = threadIdx.x;  // 0..255
     const int64_t nblk_row = args.h / kBlock;
-    int64_t qidx_base;
-    int out_off;
-    int pk_off;
+    int64_t qbase, qstep;       // q8 index of this thread's block at weight K-step kb: qbase + kb*qstep
+    int out_off, pk_off, swz;
     bool valid;
     if (!kBwd) {
       // row p of the N tile is Wt row n0 + p; its block kb is K-step kb
       const int64_t j = n0 + p;
       valid = j < args.N;
-      qidx_base = j * nblk_row;
+      qbase = j * nblk_row;
+      qstep = 1;
       pk_off = p * 32;
       out_off = (p >> 3) * 1024 + (p & 7) * 128;
+      swz = p & 7;
     } else {
       // K row jl of the stage is Wt row kb*64 + jl; column atom a is blocks n0/64 + a
       const int jl = p & 63, a = p >> 6;
       valid = (n0 + a * 64) < args.N;
-      qidx_base = (n0 / 64) + a;
+      qbase = static_cast<int64_t>(jl) * nblk_row + (n0 / 64) + a;
+      qstep = 64 * nblk_row;
       pk_off = a * 2048 + jl * 32;
       out_off = a * 8192 + (jl >> 3) * 1024 + (jl & 7) * 128;
+      swz = jl & 7;
     }
-    const int swz = (!kBwd ? p : (p & 63)) & 7;
-    for (int i = 0; i < total; ++i) {
+    // 8-bit scale and second-level scale of this thread's block, fetched two stages ahead
+    const int nk = args.num_kb;
+    uint32_t q_cur = 0u, q_nxt = 0u;
+    float s_cur = 0.f, s_nxt = 0.f;
+    if (valid && nk > 0) {
+      q_cur = __ldg(args.q8 + qbase);
+      s_cur = __ldg(args.s2 + (qbase >> 8));
+    }
+    if (valid && nk > 1) {
+      const int64_t qi = qbase + qstep;
+      q_nxt = __ldg(args.q8 + qi);
+      s_nxt = __ldg(args.s2 + (qi >> 8));
+    }
+    const int hsel = (p >> 2) & 1;  // stagger the two 16-byte halves: no bank conflicts
+    bool ok = true;
+    for (int i = 0; i < total && ok; ++i) {
       const int slot = i % STAGES;
       const uint32_t ph = (i / STAGES) & 1;
-      float k = 0.f;
-      if (i >= args.num_lkb && valid) {
-        const int kb = i - args.num_lkb;
-        const int64_t qi = !kBwd ? qidx_base + kb
-                                 : (static_cast<int64_t>(kb) * 64 + (p & 63)) * nblk_row + qidx_base;
-        k = __fmul_rn(static_cast<float>(__ldg(args.q8 + qi)), __ldg(args.s2 + (qi >> 8)));
-      }
-      if (!mbar_wait(&empty[slot], ph ^ 1u, abort_flag)) break;
+      if (!mbar_wait(&empty[slot], ph ^ 1u, abort_flag)) { ok = false; break; }
       if (i >= args.num_lkb) {
-        if (!mbar_wait(&full_ap[slot], ph, abort_flag)) break;
+        const int kb = i - args.num_lkb;
+        const float k = __fmul_rn(static_cast<float>(q_cur), s_cur);
+        q_cur = q_nxt;
+        s_cur = s_nxt;
+        if (valid && kb + 2 < nk) {
+          const int64_t qi = qbase + static_cast<int64_t>(kb + 2) * qstep;
+          q_nxt = __ldg(args.q8 + qi);
+          s_nxt = __ldg(args.s2 + (qi >> 8));
+        }
+        if (!mbar_wait(&full_ap[slot], ph, abort_flag)) { ok = false; break; }
         if (valid) {
+          uint64_t kk;
+          asm("mov.b64 %0, {%1, %1};" : "=l"(kk) : "f"(k));
           const uint4* src = reinterpret_cast<const uint4*>(sP + slot * P_BYTES + pk_off);
-          const uint4 c0 = src[0], c1 = src[1];
-          const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          const uint4 c0 = src[hsel], c1 = src[hsel ^ 1];
+          const uint4 lo = hsel ? c1 : c0, hi = hsel ? c0 : c1;
+          const uint32_t words[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
           uint8_t* dst = sB + slot * B_BYTES + out_off;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint32_t x = words[c];
-            uint4 o;
-            o.x = pack_bf16x2(__fmul_rn(lv[(x >> 4) & 15u], k), __fmul_rn(lv[x & 15u], k));
-            o.y = pack_bf16x2(__fmul_rn(lv[(x >> 12) & 15u], k), __fmul_rn(lv[(x >> 8) & 15u], k));
-            o.z = pack_bf16x2(__fmul_rn(lv[(x >> 20) & 15u], k), __fmul_rn(lv[(x >> 16) & 15u], k));
-            o.w = pack_bf16x2(__fmul_rn(lv[(x >> 28) & 15u], k), __fmul_rn(lv[(x >> 24) & 15u], k));
-            *reinterpret_cast<uint4*>(dst + ((c ^ swz) << 4)) = o;
-          }
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(dst + ((c ^ swz) << 4)) = dequant8(words[c], kk, lv);
         }
         fence_proxy_async_smem();
       }
       mbar_arrive(&full_b[slot]);
     }
-  } else if (warp < kEpiWarps) {
+
     // ---------------- epilogue: TMEM -> registers -> bf16 -> global -------------------------
-    const bool ok = mbar_wait(acc_full, 0, abort_flag);
+    const bool done = mbar_wait(acc_full, 0, abort_flag);
     tc_fence_after();
-    if (ok && !*abort_flag) {
-      const int row = m0 + warp * 32 + lane;
-      const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+    if (done && !*abort_flag) {
+      const int half = warp >> 2, quad = warp & 3;
+      const int row = m0 + half * 128 + quad * 32 + lane;
+      const uint32_t lane_addr =
+          tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(half * BN);
       for (int c = 0; c < BN / 16; ++c) {
         if (n0 + c * 16 >= args.N) break;  // N is a multiple of 64: whole chunks only
         uint32_t v[16];

@@ -590,7 +590,7 @@ int qlora_linear_fwd(const uint16_t* X, int64_t t, const nf4_weight* W, const ui
   ga.num_lkb = static_cast<int>((r + 63) / 64);
   ga.out = Y;
   ga.tab = device_table();
-  dim3 grid(static_cast<unsigned>((o + 255) / 256), static_cast<unsigned>((t + 127) / 128));
+  dim3 grid(static_cast<unsigned>((o + 255) / 256), static_cast<unsigned>((t + tc::BM - 1) / tc::BM));
   {
     prof::Scope ps(prof::kGemmFwd, st);
     nf4_gemm_kernel<false><<<grid, tc::kThreads, tc::nf4_gemm_smem_bytes(), st>>>(mA, mP, mA2,
@@ -655,7 +655,7 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t t, const nf4
     ga.num_lkb = static_cast<int>((r + 63) / 64);
     ga.out = dX;
     ga.tab = device_table();
-    dim3 grid(static_cast<unsigned>((h + 255) / 256), static_cast<unsigned>((t + 127) / 128));
+    dim3 grid(static_cast<unsigned>((h + 255) / 256), static_cast<unsigned>((t + tc::BM - 1) / tc::BM));
     {
       prof::Scope ps(prof::kGemmBwd, st);
       nf4_gemm_kernel<true><<<grid, tc::kThreads, tc::nf4_gemm_smem_bytes(), st>>>(mA, mP, mA2,
