@@ -49,7 +49,7 @@ SIGNATURES = {
     "qlora_linear_fwd_noalloc": (ctypes.c_int, [_PTR, _I64, _PTR, _PTR, _PTR, _I64,
                                                 ctypes.c_float, _PTR, _PTR, _PTR]),
 }
-KERNEL_KINDS = 8
+KERNEL_KINDS = 7
 
 
 class NF4WeightDesc(ctypes.Structure):

@@ -345,21 +345,33 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 
 // ------------------------------------------------------------------------------------------
 // Plain TMA-fed tcgen05 GEMM for the rank-r products.
-// D (M x Ncols) = alpha * A (M x K) . B (K x Ncols), Ncols <= 256 (one N tile), split-K over
+// D (M x Ncols) = A (M x K) . B (K x Ncols), Ncols <= 256 (one N tile), split-K over
 // blockIdx.z. A_MN / B_MN select MN-major operands (the TMA boxes are 64 x 64 atoms then).
+// The pipeline depth is chosen by the host from the B tile size.
 // ------------------------------------------------------------------------------------------
 namespace tcg {
-constexpr int BM = 128, BK = 64, STAGES = 4;
+constexpr int BM = 128, BK = 64, MAX_STAGES = 8;
 constexpr int A_BYTES = BM * BK * 2;        // 16 KB
-constexpr int B_MAX_BYTES = 256 * BK * 2;   // 32 KB
 constexpr int kThreads = 6 * 32;            // warps 0-3 epilogue, 4 TMA, 5 MMA
 constexpr int kTmaWarp = 4, kMmaWarp = 5;
-constexpr size_t smem_bytes() { return 1024 + STAGES * (A_BYTES + B_MAX_BYTES) + 256; }
+constexpr int kMaxSmem = 232448 - 1024;     // opt-in maximum per CTA on sm_100, less static smem
+// B tile bytes for a given MMA N (BNp, multiple of 16) and major-ness
+__host__ __device__ constexpr int b_bytes(int BNp, bool b_mn) {
+  return b_mn ? ((BNp + 63) / 64) * 8192 : BNp * 128;
+}
+__host__ __device__ constexpr int stage_bytes(int BNp, bool b_mn) {
+  return A_BYTES + ((b_bytes(BNp, b_mn) + 1023) / 1024) * 1024;
+}
+constexpr size_t smem_bytes(int stages, int BNp, bool b_mn) {
+  return 1024 + static_cast<size_t>(stages) * stage_bytes(BNp, b_mn) + 256;
+}
 }  // namespace tcg
 
 enum TcOutMode : int {
-  kOutAtomicRowMajor = 0,   // out32[m * ld + n] += alpha * acc
-  kOutAtomicTransposed = 1, // out32[n * ld + m] += alpha * acc
+  kOutAtomicRowMajor = 0,   // out32[m * ld + n] += acc
+  kOutAtomicTransposed = 1, // out32[n * ld + m] += acc
+  kOutRoundBf16 = 2,        // out32 (m * Ncols + n) += acc; the last CTA of each M tile then
+                            // writes bf16(alpha * out32) to out16a (and out16b if set)
 };
 
 struct TcGemmArgs {
@@ -368,11 +380,34 @@ struct TcGemmArgs {
   int BNp;           // MMA N: Ncols rounded up to a multiple of 16
   int num_kb;        // ceil(K / 64)
   int kb_per_split;
+  int splits;        // gridDim.z
+  int stages;
   float alpha;
   int out_mode;
   float* out32;
   int64_t ld;
+  uint16_t* out16a;
+  uint16_t* out16b;
+  unsigned* counters;  // kOutRoundBf16: one per M tile, zeroed by the caller
 };
+
+#ifdef QLORA_TRACE
+constexpr int kTraceCtas = 8192;
+__device__ unsigned long long g_trace[kTraceCtas][8];
+__device__ __forceinline__ void trace_stamp(int slot) {
+  const unsigned cta = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+  if (cta < kTraceCtas) g_trace[cta][slot] = global_timer_ns();
+}
+#define QLORA_STAMP(i) trace_stamp(i)
+#else
+#define QLORA_STAMP(i)
+#endif
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
 
 template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(tcg::kThreads, 1)
@@ -380,13 +415,15 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
                    const TcGemmArgs args) {
   using namespace tcg;
   extern __shared__ uint8_t smem_raw[];
+  __shared__ uint32_t last_flag;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = sA + STAGES * A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_MAX_BYTES);
-  uint64_t* empty = full + STAGES;
-  uint64_t* acc_full = empty + STAGES;
+  const int BNp = args.BNp;
+  const int STAGES = args.stages;
+  const int SB = stage_bytes(BNp, B_MN);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * SB);
+  uint64_t* empty = full + MAX_STAGES;
+  uint64_t* acc_full = empty + MAX_STAGES;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
   volatile uint32_t* abort_flag = tmem_holder + 1;
 
@@ -395,13 +432,12 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
   const int kb0 = blockIdx.z * args.kb_per_split;
   const int kb1 = min(args.num_kb, kb0 + args.kb_per_split);
   const int nk = kb1 - kb0;
-  const int BNp = args.BNp;
   const uint32_t tmem_cols = BNp <= 32 ? 32u : (BNp <= 64 ? 64u : (BNp <= 128 ? 128u : 256u));
   const int b_atoms = (BNp + 63) / 64;
-  const uint32_t b_bytes = B_MN ? static_cast<uint32_t>(b_atoms) * 8192u
-                                : static_cast<uint32_t>(BNp) * 128u;
+  const uint32_t bbytes = static_cast<uint32_t>(b_bytes(BNp, B_MN));
 
   if (threadIdx.x == 0) {
+    QLORA_STAMP(0);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -422,6 +458,7 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  if (threadIdx.x == 0) QLORA_STAMP(1);
 
   if (warp == kTmaWarp) {
     if (lane == 0) {
@@ -431,21 +468,22 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
         const uint32_t ph = (i / STAGES) & 1;
         if (!mbar_wait(&empty[slot], ph ^ 1u, abort_flag)) break;
         const int kb = kb0 + i;
-        mbar_arrive_expect_tx(&full[slot], A_BYTES + b_bytes);
-        uint8_t* a_dst = sA + slot * A_BYTES;
+        mbar_arrive_expect_tx(&full[slot], A_BYTES + bbytes);
+        uint8_t* a_dst = smem + slot * SB;
         if (!A_MN) {
           tma_load_2d(a_dst, &tmA, &full[slot], kb * BK, m0);
         } else {
           tma_load_2d(a_dst, &tmA, &full[slot], m0, kb * BK);
           tma_load_2d(a_dst + 8192, &tmA, &full[slot], m0 + 64, kb * BK);
         }
-        uint8_t* b_dst = sB + slot * B_MAX_BYTES;
+        uint8_t* b_dst = a_dst + A_BYTES;
         if (!B_MN) {
           tma_load_2d(b_dst, &tmB, &full[slot], kb * BK, 0);
         } else {
           for (int a = 0; a < b_atoms; ++a)
             tma_load_2d(b_dst + a * 8192, &tmB, &full[slot], a * 64, kb * BK);
         }
+        if (i == 0) QLORA_STAMP(2);
         issued = i + 1;
       }
       if (*abort_flag) {
@@ -461,9 +499,11 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
         const int slot = i % STAGES;
         const uint32_t ph = (i / STAGES) & 1;
         if (!mbar_wait(&full[slot], ph, abort_flag)) break;
+        if (i == 0) QLORA_STAMP(3);
+        if (i == nk - 1) QLORA_STAMP(4);
         tc_fence_after();
-        const uint32_t a_addr = smem_addr(sA + slot * A_BYTES);
-        const uint32_t b_addr = smem_addr(sB + slot * B_MAX_BYTES);
+        const uint32_t a_addr = smem_addr(smem + slot * SB);
+        const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
           const uint64_t ad = A_MN ? sw128_desc(a_addr + kk * 2048, 8192, 1024)
@@ -478,31 +518,67 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
       umma_commit(acc_full);
       if (*abort_flag && any) mbar_drain(acc_full, 0);
     }
-  } else if (warp < 4) {
+  } else {
+    // ---------------- epilogue warps 0-3: one accumulator row per thread ------------------
     const bool ok = (nk > 0) && mbar_wait(acc_full, 0, abort_flag);
+    if (threadIdx.x == 0) QLORA_STAMP(5);
     tc_fence_after();
     if (ok && !*abort_flag) {
       const int row = m0 + warp * 32 + lane;
       const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
-      for (int c = 0; c < BNp / 16; ++c) {
-        uint32_t v[16];
-        tmem_ld_16(lane_addr + c * 16, v);
-        tmem_ld_wait();
-        if (row < args.M) {
+      const bool direct_bf16 = args.out_mode == kOutRoundBf16 && args.splits == 1;
+      // one accumulator chunk of 16 columns -> the output mode's destination
+      auto emit = [&](const uint32_t (&v)[16], int n0) {
+        if (row >= args.M || n0 >= args.Ncols) return;  // Ncols is a multiple of 16
+        if (args.out_mode == kOutAtomicTransposed) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int n = c * 16 + e;
-            if (n < args.Ncols) {
-              const float val = args.alpha * __uint_as_float(v[e]);
-              float* dst = args.out_mode == kOutAtomicRowMajor
-                               ? args.out32 + static_cast<int64_t>(row) * args.ld + n
-                               : args.out32 + static_cast<int64_t>(n) * args.ld + row;
-              atomicAdd(dst, val);
-            }
+          for (int e = 0; e < 16; ++e)
+            atomicAdd(args.out32 + static_cast<int64_t>(n0 + e) * args.ld + row,
+                      __uint_as_float(v[e]));
+        } else if (direct_bf16) {
+          const float a = args.alpha;
+          uint4 o0, o1;
+          o0.x = pack_bf16x2(a * __uint_as_float(v[0]), a * __uint_as_float(v[1]));
+          o0.y = pack_bf16x2(a * __uint_as_float(v[2]), a * __uint_as_float(v[3]));
+          o0.z = pack_bf16x2(a * __uint_as_float(v[4]), a * __uint_as_float(v[5]));
+          o0.w = pack_bf16x2(a * __uint_as_float(v[6]), a * __uint_as_float(v[7]));
+          o1.x = pack_bf16x2(a * __uint_as_float(v[8]), a * __uint_as_float(v[9]));
+          o1.y = pack_bf16x2(a * __uint_as_float(v[10]), a * __uint_as_float(v[11]));
+          o1.z = pack_bf16x2(a * __uint_as_float(v[12]), a * __uint_as_float(v[13]));
+          o1.w = pack_bf16x2(a * __uint_as_float(v[14]), a * __uint_as_float(v[15]));
+          const int64_t off = static_cast<int64_t>(row) * args.Ncols + n0;
+          reinterpret_cast<uint4*>(args.out16a + off)[0] = o0;
+          reinterpret_cast<uint4*>(args.out16a + off)[1] = o1;
+          if (args.out16b) {
+            reinterpret_cast<uint4*>(args.out16b + off)[0] = o0;
+            reinterpret_cast<uint4*>(args.out16b + off)[1] = o1;
           }
+        } else {
+          float* dst = args.out32 + static_cast<int64_t>(row) * args.ld + n0;
+#pragma unroll
+          for (int e = 0; e < 16; e += 4)
+            red_add_v4(dst + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                       __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
         }
+      };
+      // up to four 16-column TMEM loads in flight before one wait (the counts are warp-uniform)
+      const int nchunks = BNp / 16;
+      for (int c = 0; c < nchunks; c += 4) {
+        uint32_t v0[16], v1[16], v2[16], v3[16];
+        tmem_ld_16(lane_addr + c * 16, v0);
+        if (c + 1 < nchunks) tmem_ld_16(lane_addr + (c + 1) * 16, v1);
+        if (c + 2 < nchunks) tmem_ld_16(lane_addr + (c + 2) * 16, v2);
+        if (c + 3 < nchunks) tmem_ld_16(lane_addr + (c + 3) * 16, v3);
+        tmem_ld_wait();
+        emit(v0, c * 16);
+        if (c + 1 < nchunks) emit(v1, (c + 1) * 16);
+        if (c + 2 < nchunks) emit(v2, (c + 2) * 16);
+        if (c + 3 < nchunks) emit(v3, (c + 3) * 16);
       }
+      // partial sums must be visible device-wide before this CTA is counted as arrived
+      if (args.out_mode == kOutRoundBf16 && args.splits > 1) __threadfence();
     }
+    if (threadIdx.x == 0) QLORA_STAMP(6);
   }
   tc_fence_before();
   __syncthreads();
@@ -510,6 +586,43 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, tmem_cols);
   }
+  // kOutRoundBf16 with split-K: the last CTA of this M tile to finish converts the summed
+  // fp32 rows to bf16(alpha * sum). Nobody waits on anybody: earlier CTAs just exit.
+  if (args.out_mode == kOutRoundBf16 && args.splits > 1 && nk > 0) {
+    if (threadIdx.x == 0) {
+      __threadfence();
+      const unsigned prev = atomicAdd(args.counters + blockIdx.y, 1u);
+      last_flag = (prev == static_cast<unsigned>(args.splits - 1)) ? 1u : 0u;
+      __threadfence();
+    }
+    __syncthreads();
+    if (last_flag && warp < 4 && !*abort_flag) {
+      const int row = m0 + warp * 32 + lane;
+      if (row < args.M) {
+        const float* src = args.out32 + static_cast<int64_t>(row) * args.Ncols;
+        uint16_t* da = args.out16a + static_cast<int64_t>(row) * args.Ncols;
+        uint16_t* db = args.out16b ? args.out16b + static_cast<int64_t>(row) * args.Ncols : nullptr;
+        // 64 columns (16 independent 16-byte loads) in flight per round
+        for (int n0 = 0; n0 < args.Ncols; n0 += 64) {
+          float4 x[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u)
+            if (n0 + 4 * u < args.Ncols)
+              x[u] = __ldcg(reinterpret_cast<const float4*>(src + n0 + 4 * u));
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            if (n0 + 4 * u >= args.Ncols) break;
+            uint2 o;
+            o.x = pack_bf16x2(args.alpha * x[u].x, args.alpha * x[u].y);
+            o.y = pack_bf16x2(args.alpha * x[u].z, args.alpha * x[u].w);
+            *reinterpret_cast<uint2*>(da + n0 + 4 * u) = o;
+            if (db) *reinterpret_cast<uint2*>(db + n0 + 4 * u) = o;
+          }
+        }
+      }
+    }
+  }
+  if (threadIdx.x == 0) QLORA_STAMP(7);
 }
 
 }  // namespace qlora

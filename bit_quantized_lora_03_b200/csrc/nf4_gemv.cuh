@@ -133,36 +133,22 @@ __global__ void __launch_bounds__(128) nf4_gemv_kernel(const GemvArgs args) {
       }
 }
 
-// Y[n][j] = bf16( Y32[n][j] + sum_c sT[n][c] * L2[c][j] ), sT = bf16(s * T32): the LoRA
+// Y[n][j] = bf16( Y32[n][j] + sum_c sT[n][c] * L2[c][j] ) with sT = bf16(s . X.L1): the LoRA
 // up-projection folded into the GEMV's output conversion. Grid (ceil(o/256), t).
 __global__ void __launch_bounds__(256) gemv_lora_finalize_kernel(
-    const float* __restrict__ Y32, const float* __restrict__ T32, const uint16_t* __restrict__ L2,
-    uint16_t* __restrict__ Y, int64_t o, int r, float s) {
-  __shared__ float sT[256];
+    const float* __restrict__ Y32, const uint16_t* __restrict__ sT, const uint16_t* __restrict__ L2,
+    uint16_t* __restrict__ Y, int64_t o, int r) {
+  __shared__ float sTs[256];
   const int n = blockIdx.y;
   for (int c = threadIdx.x; c < r; c += blockDim.x)
-    sT[c] = bf16_bits_to_float(__bfloat16_as_ushort(
-        __float2bfloat16_rn(__fmul_rn(s, T32[static_cast<int64_t>(n) * r + c]))));
+    sTs[c] = bf16_bits_to_float(sT[static_cast<int64_t>(n) * r + c]);
   __syncthreads();
   const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (j >= o) return;
   float y = Y32[static_cast<int64_t>(n) * o + j];
   for (int c = 0; c < r; ++c)
-    y = fmaf(sT[c], bf16_bits_to_float(L2[static_cast<int64_t>(c) * o + j]), y);
+    y = fmaf(sTs[c], bf16_bits_to_float(L2[static_cast<int64_t>(c) * o + j]), y);
   Y[static_cast<int64_t>(n) * o + j] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
-}
-
-// sT[m][c] = bf16(s * T32[m][c]) (the saved LoRA down-projection, also the A operand of the
-// folded LoRA K-steps of the fused GEMM). Elementwise over t*r.
-__global__ void __launch_bounds__(256) lora_scale_round_kernel(const float* __restrict__ T32,
-                                                               uint16_t* __restrict__ out_a,
-                                                               uint16_t* __restrict__ out_b,
-                                                               int64_t count, float s) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= count) return;
-  const uint16_t v = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(s, T32[i])));
-  if (out_a) out_a[i] = v;
-  if (out_b) out_b[i] = v;
 }
 
 }  // namespace qlora

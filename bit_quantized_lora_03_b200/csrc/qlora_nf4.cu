@@ -8,6 +8,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -122,13 +123,13 @@ int current_device(int* dev_out) {
                                  static_cast<int>(tc::nf4_gemm_smem_bytes())) == cudaSuccess;
     fine &= cudaFuncSetAttribute(tc_gemm_kernel<false, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(tcg::smem_bytes())) == cudaSuccess;
+                                 tcg::kMaxSmem) == cudaSuccess;
     fine &= cudaFuncSetAttribute(tc_gemm_kernel<false, true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(tcg::smem_bytes())) == cudaSuccess;
+                                 tcg::kMaxSmem) == cudaSuccess;
     fine &= cudaFuncSetAttribute(tc_gemm_kernel<true, true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(tcg::smem_bytes())) == cudaSuccess;
+                                 tcg::kMaxSmem) == cudaSuccess;
     if (!fine) cudaGetLastError();
     d.ok = fine ? 1 : -1;
   });
@@ -149,11 +150,11 @@ int launch_status() {
 // ------------------------------------------------------------------------------------------
 namespace prof {
 enum Kind {
-  kQuant = 0, kDequant, kGemv, kGemvFinalize, kScaleRound, kTcGemm, kGemmFwd, kGemmBwd, kKinds
+  kQuant = 0, kDequant, kGemv, kGemvFinalize, kTcGemm, kGemmFwd, kGemmBwd, kKinds
 };
 const char* const kNames[kKinds] = {
     "nf4_quantize_kernel", "nf4_dequantize_kernel", "nf4_gemv_kernel",
-    "gemv_lora_finalize_kernel", "lora_scale_round_kernel", "tc_gemm_kernel",
+    "gemv_lora_finalize_kernel", "tc_gemm_kernel",
     "nf4_gemm_kernel<fwd>", "nf4_gemm_kernel<bwd>"};
 static_assert(kKinds == QLORA_KERNEL_KINDS, "kernel kinds");
 
@@ -265,9 +266,13 @@ int check_linear_shape(int64_t t, int64_t h, int64_t o, int64_t r) {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// workspace regions (each 256-byte aligned): fp32 t x r accumulator, bf16 t x r
+// workspace region of one rank-r down projection (each part 256-byte aligned): the fp32
+// t x r split-K accumulator, one arrival counter per 128-token tile (zeroed together with the
+// accumulator), and the bf16 t x r result
+size_t lora_acc_bytes(int64_t t, int64_t r) { return align256(static_cast<size_t>(t) * r * 4); }
+size_t lora_counter_bytes(int64_t t) { return align256(static_cast<size_t>((t + 127) / 128) * 4); }
 size_t lora_region_bytes(int64_t t, int64_t r) {
-  return align256(static_cast<size_t>(t) * r * 4) + align256(static_cast<size_t>(t) * r * 2);
+  return lora_acc_bytes(t, r) + lora_counter_bytes(t) + align256(static_cast<size_t>(t) * r * 2);
 }
 
 // fp32 t x o accumulator for the GEMV's split-K partial sums
@@ -280,70 +285,102 @@ constexpr int64_t kGemvMaxTokens = 16;
 // ------------------------------------------------------------------------------------------
 // launch helpers
 // ------------------------------------------------------------------------------------------
-int splits_for(int ctas, int num_kb, int sms) {
-  int s = std::max(1, (sms + ctas - 1) / std::max(1, ctas));
-  s = std::min(s, num_kb);
-  return std::max(1, s);
+struct TcPlan {
+  int stages, splits, kb_per_split, num_kb, mtiles, BNp;
+  size_t smem;
+};
+
+// These products stream one large operand (X or dY, read once from HBM) through a small
+// accumulator. One wave of one CTA per SM, each with the deepest pipeline that fits (up to 8
+// stages), keeps HBM busy; split-K only as far as needed to give every SM a CTA, so the fixed
+// per-CTA costs (set-up, epilogue, the final rounding) are paid as few times as possible.
+TcPlan plan_tc(int64_t M, int64_t ncols, int64_t K, bool b_mn, int sms) {
+  TcPlan p{};
+  p.BNp = static_cast<int>((ncols + 15) / 16 * 16);
+  p.num_kb = static_cast<int>((K + 63) / 64);
+  p.mtiles = static_cast<int>((M + 127) / 128);
+  int stages = tcg::MAX_STAGES;
+  while (stages > 2 && tcg::smem_bytes(stages, p.BNp, b_mn) > static_cast<size_t>(tcg::kMaxSmem))
+    --stages;
+  p.stages = stages;
+  p.smem = tcg::smem_bytes(stages, p.BNp, b_mn);
+  int splits = std::max(1, sms / p.mtiles);
+  splits = std::min(splits, std::max(1, p.num_kb / 4));
+#ifdef QLORA_TUNING
+  if (const char* e = std::getenv("QLORA_TC_WAVE")) splits = std::max(1, (std::atoi(e) * sms) / p.mtiles);
+  if (const char* e = std::getenv("QLORA_TC_MINKB")) splits = std::min(splits, std::max(1, p.num_kb / std::atoi(e)));
+  if (const char* e = std::getenv("QLORA_TC_STAGES")) {
+    p.stages = std::atoi(e);
+    p.smem = tcg::smem_bytes(p.stages, p.BNp, b_mn);
+  }
+#endif
+  p.kb_per_split = (p.num_kb + splits - 1) / splits;
+  p.splits = (p.num_kb + p.kb_per_split - 1) / p.kb_per_split;
+  return p;
 }
 
-// D (M x ncols) += alpha * A . B with the generic tcgen05 GEMM, split-K so the grid fills the
-// GPU. Output fp32 by atomic adds (caller zeroes it).
 template <bool A_MN, bool B_MN>
 int launch_tc_gemm(const CUtensorMap& mA, const CUtensorMap& mB, int64_t M, int64_t ncols,
-                   int64_t K, float alpha, int mode, float* out32, int64_t ld, int sms,
-                   cudaStream_t st) {
+                   const TcPlan& pl, float alpha, int mode, float* out32, int64_t ld,
+                   uint16_t* o16a, uint16_t* o16b, unsigned* counters, cudaStream_t st) {
   TcGemmArgs a{};
   a.M = static_cast<int>(M);
   a.Ncols = static_cast<int>(ncols);
-  a.BNp = static_cast<int>((ncols + 15) / 16 * 16);
-  a.num_kb = static_cast<int>((K + 63) / 64);
-  const int mtiles = static_cast<int>((M + 127) / 128);
-  const int splits = splits_for(mtiles, a.num_kb, sms);
-  a.kb_per_split = (a.num_kb + splits - 1) / splits;
-  const int zs = (a.num_kb + a.kb_per_split - 1) / a.kb_per_split;
+  a.BNp = pl.BNp;
+  a.num_kb = pl.num_kb;
+  a.kb_per_split = pl.kb_per_split;
+  a.splits = pl.splits;
+  a.stages = pl.stages;
   a.alpha = alpha;
   a.out_mode = mode;
   a.out32 = out32;
   a.ld = ld;
-  dim3 grid(1, mtiles, zs);
+  a.out16a = o16a;
+  a.out16b = o16b;
+  a.counters = counters;
+  dim3 grid(1, pl.mtiles, pl.splits);
   {
     prof::Scope ps(prof::kTcGemm, st);
-    tc_gemm_kernel<A_MN, B_MN><<<grid, tcg::kThreads, tcg::smem_bytes(), st>>>(mA, mB, a);
+    tc_gemm_kernel<A_MN, B_MN><<<grid, tcg::kThreads, pl.smem, st>>>(mA, mB, a);
   }
   return launch_status();
 }
 
 struct LoraWs {
-  float* acc32;   // t x r fp32
-  uint16_t* b16;  // t x r bf16
+  float* acc32;        // t x r fp32
+  unsigned* counters;  // one per 128-token tile
+  uint16_t* b16;       // t x r bf16
 };
 
 LoraWs carve_lora(void* base, int64_t t, int64_t r) {
   LoraWs w;
-  w.acc32 = reinterpret_cast<float*>(base);
-  w.b16 = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(base) +
-                                      align256(static_cast<size_t>(t) * r * 4));
+  uint8_t* b = reinterpret_cast<uint8_t*>(base);
+  w.acc32 = reinterpret_cast<float*>(b);
+  w.counters = reinterpret_cast<unsigned*>(b + lora_acc_bytes(t, r));
+  w.b16 = reinterpret_cast<uint16_t*>(b + lora_acc_bytes(t, r) + lora_counter_bytes(t));
   return w;
 }
 
-// s . A . B^(T) for the rank-r down projections: out16 = bf16(s * A.B) (and out16b if given).
-// A is t x K (K-major), B is given by its map. Uses ws.acc32 as the fp32 accumulator.
+// out16 = bf16(s . A.B) (and out16b if given) for a rank-r down projection: A is t x K
+// (K-major), B given by its map (ncols = r). One launch; with split-K the partial sums meet
+// in ws.acc32 and the last CTA of each 128-token tile rounds them.
 template <bool B_MN>
 int lora_down(const CUtensorMap& mA, const CUtensorMap& mB, int64_t t, int64_t K, int64_t r,
               float s, const LoraWs& ws, uint16_t* out16, uint16_t* out16b, int sms,
               cudaStream_t st) {
-  if (cudaMemsetAsync(ws.acc32, 0, static_cast<size_t>(t) * r * 4, st) != cudaSuccess)
-    return QLORA_ERR_CUDA;
-  int rc = launch_tc_gemm<false, B_MN>(mA, mB, t, r, K, 1.0f, kOutAtomicRowMajor, ws.acc32, r,
-                                       sms, st);
-  if (rc) return rc;
-  const int64_t count = t * r;
-  {
-    prof::Scope ps(prof::kScaleRound, st);
-    lora_scale_round_kernel<<<static_cast<unsigned>((count + 255) / 256), 256, 0, st>>>(
-        ws.acc32, out16, out16b, count, s);
+  TcPlan pl = plan_tc(t, r, K, B_MN, sms);
+#ifdef QLORA_TUNING
+  if (const char* e = std::getenv("QLORA_RB_SPLITS")) {
+    int sp = std::max(1, std::min(pl.num_kb, std::atoi(e)));
+    pl.kb_per_split = (pl.num_kb + sp - 1) / sp;
+    pl.splits = (pl.num_kb + pl.kb_per_split - 1) / pl.kb_per_split;
   }
-  return launch_status();
+#endif
+  if (pl.splits > 1 &&
+      cudaMemsetAsync(ws.acc32, 0, lora_acc_bytes(t, r) + lora_counter_bytes(t), st) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return launch_tc_gemm<false, B_MN>(mA, mB, t, r, pl, s, kOutRoundBf16, ws.acc32, r, out16,
+                                     out16b, ws.counters, st);
 }
 
 }  // namespace
@@ -522,12 +559,9 @@ int qlora_linear_fwd(const uint16_t* X, int64_t t, const nf4_weight* W, const ui
   if (t <= kGemvMaxTokens) {
     float* Y32 = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) +
                                           lora_region_bytes(t, r));
-    if (cudaMemsetAsync(ws.acc32, 0, static_cast<size_t>(t) * r * 4, st) != cudaSuccess ||
-        cudaMemsetAsync(Y32, 0, static_cast<size_t>(t) * o * 4, st) != cudaSuccess)
+    if (cudaMemsetAsync(Y32, 0, static_cast<size_t>(t) * o * 4, st) != cudaSuccess)
       return QLORA_ERR_CUDA;
-    if ((rc = launch_tc_gemm<false, true>(mX, mL1, t, r, h, 1.0f, kOutAtomicRowMajor, ws.acc32, r,
-                                          sms, st)))
-      return rc;
+    if ((rc = lora_down<true>(mX, mL1, t, h, r, s, ws, ws.b16, sT_out, sms, st))) return rc;
     GemvArgs ga{};
     ga.codes = W->codes;
     ga.q8 = W->absmax_q8;
@@ -557,18 +591,10 @@ int qlora_linear_fwd(const uint16_t* X, int64_t t, const nf4_weight* W, const ui
     dim3 fgrid(static_cast<unsigned>((o + 255) / 256), static_cast<unsigned>(t));
     {
       prof::Scope ps(prof::kGemvFinalize, st);
-      gemv_lora_finalize_kernel<<<fgrid, 256, 0, st>>>(Y32, ws.acc32, L2, Y, o,
-                                                       static_cast<int>(r), s);
+      gemv_lora_finalize_kernel<<<fgrid, 256, 0, st>>>(Y32, ws.b16, L2, Y, o,
+                                                       static_cast<int>(r));
     }
-    if ((rc = launch_status())) return rc;
-    if (sT_out) {
-      const int64_t count = t * r;
-      prof::Scope ps(prof::kScaleRound, st);
-      lora_scale_round_kernel<<<static_cast<unsigned>((count + 255) / 256), 256, 0, st>>>(
-          ws.acc32, sT_out, nullptr, count, s);
-      if ((rc = launch_status())) return rc;
-    }
-    return QLORA_OK;
+    return launch_status();
   }
 
   uint16_t* sT = ws.b16;
@@ -672,11 +698,13 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t t, const nf4
   if (!map_bf16(&mXmn, X, h, t, 64, 64) || !map_bf16(&msU, sU, r, t, 64, 64) ||
       !map_bf16(&mdYmn, dY, o, t, 64, 64) || !map_bf16(&msT, sT, r, t, 64, 64))
     return QLORA_ERR_CUDA;
-  if ((rc = launch_tc_gemm<true, true>(mXmn, msU, h, r, t, 1.0f, kOutAtomicRowMajor, dL1, r, sms,
-                                       st)))
+  const TcPlan p1 = plan_tc(h, r, t, true, sms);
+  if ((rc = launch_tc_gemm<true, true>(mXmn, msU, h, r, p1, 1.0f, kOutAtomicRowMajor, dL1, r,
+                                       nullptr, nullptr, nullptr, st)))
     return rc;
-  return launch_tc_gemm<true, true>(mdYmn, msT, o, r, t, 1.0f, kOutAtomicTransposed, dL2, o, sms,
-                                    st);
+  const TcPlan p2 = plan_tc(o, r, t, true, sms);
+  return launch_tc_gemm<true, true>(mdYmn, msT, o, r, p2, 1.0f, kOutAtomicTransposed, dL2, o,
+                                    nullptr, nullptr, nullptr, st);
 }
 
 }  // extern "C"
@@ -737,3 +765,14 @@ extern "C" int qlora_linear_fwd_noalloc(const uint16_t* X, int64_t t, const nf4_
   return qlora_linear_fwd(X, t, W, L1, L2, r, s, Y, sT_out, scratch,
                           scratch ? static_cast<size_t>(QLORA_STATIC_SCRATCH_BYTES) : 0, stream);
 }
+
+#ifdef QLORA_TRACE
+extern "C" QLORA_API int qlora_trace_read(void* host, size_t bytes) {
+  if (bytes > sizeof(g_trace)) bytes = sizeof(g_trace);
+  return cudaMemcpyFromSymbol(host, g_trace, bytes) == cudaSuccess ? 0 : -5;
+}
+extern "C" QLORA_API int qlora_trace_clear() {
+  static unsigned long long zero[kTraceCtas][8];
+  return cudaMemcpyToSymbol(g_trace, zero, sizeof(zero)) == cudaSuccess ? 0 : -5;
+}
+#endif

@@ -191,7 +191,7 @@ QLORA_API int qlora_get_last_status(qlora_stream_t stream);
  * or QLORA_ERR_INVALID_ARG if the profile overflowed its capacity. Kinds are numbered
  * 0 .. QLORA_KERNEL_KINDS-1 and named by qlora_kernel_name. Not thread-safe across
  * concurrent calls into the library while open. */
-#define QLORA_KERNEL_KINDS 8
+#define QLORA_KERNEL_KINDS 7
 QLORA_API int qlora_profile_begin(int capacity);
 QLORA_API int qlora_profile_end(double *ms, int64_t *launches, int nkinds);
 QLORA_API const char *qlora_kernel_name(int kind);
