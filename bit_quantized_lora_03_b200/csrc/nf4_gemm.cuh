@@ -9,11 +9,12 @@
 //    A (X or dY) and the packed codes arrive by TMA; 8 producer warps turn each 64-weight
 //    block into bf16 (w' = bf16(level * (q8 * s2)), the exact nf4_dequantize values) and
 //    write it straight into the 128-byte-swizzled operand layout the MMA reads: K-major for
-//    the forward (rows of Wt are N), MN-major for the backward (rows of Wt are K). A CTA owns
-//    256 tokens x 256 columns: one thread issues tcgen05.mma into two 128 x 256 fp32
-//    accumulators in tensor memory (all 512 columns), so every dequantized weight tile feeds
-//    256 tokens. The r/64 LoRA K-steps (A = sT or sU, B = L2 or L1, both by TMA) run first,
-//    then the h/64 (or o/64) weight K-steps. The same 8 warps then drain TMEM to bf16.
+//    the forward (rows of Wt are N), MN-major for the backward (rows of Wt are K). A pair of
+//    CTAs (a cluster of 2) owns 512 tokens x 256 columns and issues tcgen05.mma.cta_group::2:
+//    each CTA dequantizes only its 128 of the 256 columns, and two accumulators per CTA (all
+//    512 TMEM columns) make every dequantized tile feed 512 tokens. The r/64 LoRA K-steps
+//    (A = sT or sU, B = L2 or L1, both by TMA) run first, then the h/64 (or o/64) weight
+//    K-steps. The same 8 warps then drain TMEM to bf16.
 //
 // 2) tc_gemm_kernel<A_MN, B_MN>: a plain TMA-fed tcgen05 GEMM (both operands by TMA, either
 //    major-ness) with split-K and fp32 atomic or bf16 output, for the rank-r products
@@ -28,17 +29,23 @@
 namespace qlora {
 namespace tc {
 
-constexpr int BM = 256;        // tokens per tile: two 128-lane TMEM accumulators
-constexpr int BN = 256;        // output columns per tile (fp32 TMEM columns per accumulator)
+// A CTA pair (thread-block cluster of 2) owns 512 tokens x 256 output columns. One
+// tcgen05.mma.cta_group::2 computes 256 tokens x 256 columns: each CTA supplies 128 rows of A
+// and 128 of the 256 columns of B from its own shared memory and holds its 128 x 256 fp32
+// slice of the accumulator in its own tensor memory. Two such accumulators per CTA (all 512
+// TMEM columns) cover the 512 tokens, so each dequantized half-tile feeds 512 tokens.
+constexpr int PAIR_M = 512;
+constexpr int BN = 256;        // output columns per pair
+constexpr int BNH = BN / 2;    // columns of B held (and dequantized) by each CTA
 constexpr int BK = 64;         // K per stage: one 128-byte swizzle row of bf16, one NF4 block
-constexpr int STAGES = 3;
-constexpr int A_HALF = 128 * BK * 2;       // 16 KB: one 128-token half of the A tile
-constexpr int A_BYTES = BM * BK * 2;       // 32 KB
-constexpr int B_BYTES = BN * BK * 2;       // 32 KB
-constexpr int P_BYTES = BN * BK / 2;       // 8 KB of packed codes
+constexpr int STAGES = 4;
+constexpr int A_HALF = 128 * BK * 2;       // 16 KB: this CTA's 128 rows of one accumulator
+constexpr int A_BYTES = 2 * A_HALF;        // 32 KB
+constexpr int B_BYTES = BNH * BK * 2;      // 16 KB
+constexpr int P_BYTES = BNH * BK / 2;      // 4 KB of packed codes
 constexpr int kWorkWarps = 8;              // warps 0-7: dequant producers, then epilogue
 constexpr int kTmaWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kMmaWarp = 9;                // even CTA: MMA issuer; odd CTA: readiness relay
 constexpr int kThreads = 10 * 32;
 constexpr int kTmemCols = 512;
 
@@ -117,20 +124,24 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   uint8_t* sP = sB + STAGES * B_BYTES;
   uint64_t* full_ap = reinterpret_cast<uint64_t*>(sP + STAGES * P_BYTES);
   uint64_t* full_b = full_ap + STAGES;
-  uint64_t* empty = full_b + STAGES;
+  uint64_t* peer_ready = full_b + STAGES;   // even CTA: the odd CTA's stage is complete
+  uint64_t* empty = peer_ready + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
   volatile uint32_t* abort_flag = tmem_holder + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN;
-  const int m0 = blockIdx.y * BM;
+  const uint32_t rank = cluster_ctarank();             // 0: MMA issuer, 1: its peer
+  const int n0 = blockIdx.y * BN;                        // the pair's 256 output columns
+  const int nh0 = n0 + static_cast<int>(rank) * BNH;    // this CTA's 128 of them
+  const int mrow = (blockIdx.x >> 1) * PAIR_M + static_cast<int>(rank) * 128;  // + a * 256
   const int total = args.num_lkb + args.num_kb;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_ap[s], 1);
       mbar_init(&full_b[s], kWorkWarps * 32);
+      mbar_init(&peer_ready[s], 1);
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
@@ -139,8 +150,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   }
   if (threadIdx.x < 16) lv[threadIdx.x] = args.tab.level[threadIdx.x];
   if (warp == kMmaWarp) {
-    tmem_alloc(tmem_holder, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc2(tmem_holder, kTmemCols);
+    tmem_relinquish2();
   }
   if (warp == kTmaWarp && lane == 0) {
     tma_prefetch_desc(&tmA);
@@ -150,6 +161,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();   // both CTAs' barriers exist before any cross-CTA arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
@@ -161,32 +173,29 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         const uint32_t ph = (i / STAGES) & 1;
         if (!mbar_wait(&empty[slot], ph ^ 1u, abort_flag)) break;
         uint8_t* a_dst = sA + slot * A_BYTES;
+        uint8_t* b_dst = sB + slot * B_BYTES;
         if (i < args.num_lkb) {
           mbar_arrive_expect_tx(&full_ap[slot], A_BYTES + B_BYTES);
-          tma_load_2d(a_dst, &tmA2, &full_ap[slot], i * BK, m0);
-          tma_load_2d(a_dst + A_HALF, &tmA2, &full_ap[slot], i * BK, m0 + 128);
+          tma_load_2d(a_dst, &tmA2, &full_ap[slot], i * BK, mrow);
+          tma_load_2d(a_dst + A_HALF, &tmA2, &full_ap[slot], i * BK, mrow + 256);
           if (!kBwd) {
-            // L2 (r x o), MN-major B: four 64-column atoms, 8 KB apart
-#pragma unroll
-            for (int a = 0; a < 4; ++a)
-              tma_load_2d(sB + slot * B_BYTES + a * 8192, &tmB2, &full_ap[slot], n0 + a * 64,
-                          i * BK);
+            // L2 (r x o), MN-major B: this CTA's two 64-column atoms, 8 KB apart
+            tma_load_2d(b_dst, &tmB2, &full_ap[slot], nh0, i * BK);
+            tma_load_2d(b_dst + 8192, &tmB2, &full_ap[slot], nh0 + 64, i * BK);
           } else {
-            // L1 (h x r), K-major B: 256 rows of 64 ranks
-            tma_load_2d(sB + slot * B_BYTES, &tmB2, &full_ap[slot], i * BK, n0);
+            // L1 (h x r), K-major B: this CTA's 128 rows of 64 ranks
+            tma_load_2d(b_dst, &tmB2, &full_ap[slot], i * BK, nh0);
           }
         } else {
           const int kb = i - args.num_lkb;
           mbar_arrive_expect_tx(&full_ap[slot], A_BYTES + P_BYTES);
-          tma_load_2d(a_dst, &tmA, &full_ap[slot], kb * BK, m0);
-          tma_load_2d(a_dst + A_HALF, &tmA, &full_ap[slot], kb * BK, m0 + 128);
+          tma_load_2d(a_dst, &tmA, &full_ap[slot], kb * BK, mrow);
+          tma_load_2d(a_dst + A_HALF, &tmA, &full_ap[slot], kb * BK, mrow + 256);
           if (!kBwd) {
-            tma_load_2d(sP + slot * P_BYTES, &tmP, &full_ap[slot], kb * (BK / 2), n0);
+            tma_load_2d(sP + slot * P_BYTES, &tmP, &full_ap[slot], kb * (BK / 2), nh0);
           } else {
-#pragma unroll
-            for (int a = 0; a < 4; ++a)
-              tma_load_2d(sP + slot * P_BYTES + a * 2048, &tmP, &full_ap[slot], n0 / 2 + a * 32,
-                          kb * BK);
+            tma_load_2d(sP + slot * P_BYTES, &tmP, &full_ap[slot], nh0 / 2, kb * BK);
+            tma_load_2d(sP + slot * P_BYTES + 2048, &tmP, &full_ap[slot], nh0 / 2 + 32, kb * BK);
           }
         }
         issued = i + 1;
@@ -198,15 +207,17 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       }
     }
   } else if (warp == kMmaWarp) {
-    if (lane == 0) {
-      constexpr uint32_t kIdescMain = idesc_bf16(128, BN, false, kBwd);
-      constexpr uint32_t kIdescLora = idesc_bf16(128, BN, false, !kBwd);
+    if (lane == 0 && rank == 0) {
+      // M = 256 per instruction (128 rows from each CTA), N = 256 (128 columns from each)
+      constexpr uint32_t kIdescMain = idesc_bf16(256, BN, false, kBwd);
+      constexpr uint32_t kIdescLora = idesc_bf16(256, BN, false, !kBwd);
       bool any = false;
       for (int i = 0; i < total; ++i) {
         const int slot = i % STAGES;
         const uint32_t ph = (i / STAGES) & 1;
         if (!mbar_wait(&full_ap[slot], ph, abort_flag)) break;
         if (!mbar_wait(&full_b[slot], ph, abort_flag)) break;
+        if (!mbar_wait_cluster(&peer_ready[slot], ph, abort_flag)) break;
         tc_fence_after();
         const bool lora = i < args.num_lkb;
         const bool b_mn = lora ? !kBwd : kBwd;
@@ -218,42 +229,52 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
           const uint64_t bd = b_mn ? sw128_desc(b_addr + kk * 2048, 8192, 1024)
                                    : sw128_desc(b_addr + kk * 32, 16, 1024);
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const uint64_t ad = sw128_desc(a_addr + half * A_HALF + kk * 32, 16, 1024);
-            umma_bf16(tmem_base + half * BN, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          for (int a = 0; a < 2; ++a) {
+            const uint64_t ad = sw128_desc(a_addr + a * A_HALF + kk * 32, 16, 1024);
+            umma2_bf16(tmem_base + a * BN, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        umma_commit(&empty[slot]);
+        umma2_commit_multicast(&empty[slot], 0x3);   // frees the stage in both CTAs
         any = true;
       }
-      // completes once every MMA above has finished (also after an abort)
-      umma_commit(acc_full);
+      // completes in both CTAs once every MMA above has finished (also after an abort)
+      umma2_commit_multicast(acc_full, 0x3);
       if (*abort_flag && any) mbar_drain(acc_full, 0);
+    } else if (lane == 0) {
+      // odd CTA: tell the issuer when this CTA's half of each stage is in shared memory
+      for (int i = 0; i < total; ++i) {
+        const int slot = i % STAGES;
+        const uint32_t ph = (i / STAGES) & 1;
+        if (!mbar_wait(&full_ap[slot], ph, abort_flag)) break;
+        if (!mbar_wait(&full_b[slot], ph, abort_flag)) break;
+        mbar_arrive_remote(&peer_ready[slot], 0);
+      }
     }
   } else {
-    // ---------------- warps 0-7: dequant producers (one 64-weight block per thread per
-    // stage), then the epilogue ---------------------------------------------------------
-    const int p = threadIdx.x;  // 0..255
+    // ---------------- warps 0-7: dequant producers (half a 64-weight block per thread per
+    // stage: 128 blocks of this CTA's 128 columns), then the epilogue -----------------------
+    const int p = threadIdx.x;       // 0..255
+    const int blk = p >> 1, half = p & 1;
     const int64_t nblk_row = args.h / kBlock;
     int64_t qbase, qstep;       // q8 index of this thread's block at weight K-step kb: qbase + kb*qstep
     int out_off, pk_off, swz;
     bool valid;
     if (!kBwd) {
-      // row p of the N tile is Wt row n0 + p; its block kb is K-step kb
-      const int64_t j = n0 + p;
+      // block row blk of this CTA's columns is Wt row nh0 + blk; its block kb is K-step kb
+      const int64_t j = nh0 + blk;
       valid = j < args.N;
       qbase = j * nblk_row;
       qstep = 1;
-      pk_off = p * 32;
-      out_off = (p >> 3) * 1024 + (p & 7) * 128;
-      swz = p & 7;
+      pk_off = blk * 32 + half * 16;
+      out_off = (blk >> 3) * 1024 + (blk & 7) * 128;
+      swz = blk & 7;
     } else {
-      // K row jl of the stage is Wt row kb*64 + jl; column atom a is blocks n0/64 + a
-      const int jl = p & 63, a = p >> 6;
-      valid = (n0 + a * 64) < args.N;
-      qbase = static_cast<int64_t>(jl) * nblk_row + (n0 / 64) + a;
+      // K row jl of the stage is Wt row kb*64 + jl; local column atom a is blocks nh0/64 + a
+      const int jl = blk & 63, a = blk >> 6;
+      valid = (nh0 + a * 64) < args.N;
+      qbase = static_cast<int64_t>(jl) * nblk_row + (nh0 / 64) + a;
       qstep = 64 * nblk_row;
-      pk_off = a * 2048 + jl * 32;
+      pk_off = a * 2048 + jl * 32 + half * 16;
       out_off = a * 8192 + (jl >> 3) * 1024 + (jl & 7) * 128;
       swz = jl & 7;
     }
@@ -270,7 +291,6 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       q_nxt = __ldg(args.q8 + qi);
       s_nxt = __ldg(args.s2 + (qi >> 8));
     }
-    const int hsel = (p >> 2) & 1;  // stagger the two 16-byte halves: no bank conflicts
     bool ok = true;
     for (int i = 0; i < total && ok; ++i) {
       const int slot = i % STAGES;
@@ -290,14 +310,14 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         if (valid) {
           uint64_t kk;
           asm("mov.b64 %0, {%1, %1};" : "=l"(kk) : "f"(k));
-          const uint4* src = reinterpret_cast<const uint4*>(sP + slot * P_BYTES + pk_off);
-          const uint4 c0 = src[hsel], c1 = src[hsel ^ 1];
-          const uint4 lo = hsel ? c1 : c0, hi = hsel ? c0 : c1;
-          const uint32_t words[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+          const uint4 c = *reinterpret_cast<const uint4*>(sP + slot * P_BYTES + pk_off);
+          const uint32_t words[4] = {c.x, c.y, c.z, c.w};
           uint8_t* dst = sB + slot * B_BYTES + out_off;
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(dst + ((c ^ swz) << 4)) = dequant8(words[c], kk, lv);
+          for (int u = 0; u < 4; ++u) {
+            const int ch = half * 4 + u;   // 16-byte chunk (8 weights) within the 128-byte row
+            *reinterpret_cast<uint4*>(dst + ((ch ^ swz) << 4)) = dequant8(words[u], kk, lv);
+          }
         }
         fence_proxy_async_smem();
       }
@@ -308,10 +328,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     const bool done = mbar_wait(acc_full, 0, abort_flag);
     tc_fence_after();
     if (done && !*abort_flag) {
-      const int half = warp >> 2, quad = warp & 3;
-      const int row = m0 + half * 128 + quad * 32 + lane;
+      const int acc = warp >> 2, quad = warp & 3;
+      const int row = mrow + acc * 256 + quad * 32 + lane;
       const uint32_t lane_addr =
-          tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(half * BN);
+          tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN);
       for (int c = 0; c < BN / 16; ++c) {
         if (n0 + c * 16 >= args.N) break;  // N is a multiple of 64: whole chunks only
         uint32_t v[16];
@@ -337,9 +357,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();   // no CTA leaves while its peer may still signal it or read its TMEM slice
   if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc2(tmem_base, kTmemCols);
   }
 }
 

@@ -361,6 +361,37 @@ LoraWs carve_lora(void* base, int64_t t, int64_t r) {
   return w;
 }
 
+// The fused NF4 GEMM runs as clusters of 2 CTAs (cta_group::2): grid x = 2 CTAs per 512 tokens,
+// grid y = 256-column tiles.
+template <bool kBwd>
+int launch_nf4_gemm(const CUtensorMap& mA, const CUtensorMap& mP, const CUtensorMap& mA2,
+                    const CUtensorMap& mB2, const Nf4GemmArgs& ga, int64_t t, int64_t ncols,
+                    cudaStream_t st, int prof_kind) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * ((t + tc::PAIR_M - 1) / tc::PAIR_M)),
+                     static_cast<unsigned>((ncols + tc::BN - 1) / tc::BN), 1);
+  cfg.blockDim = dim3(tc::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = tc::nf4_gemm_smem_bytes();
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
+  {
+    prof::Scope ps(prof_kind, st);
+    e = cudaLaunchKernelEx(&cfg, nf4_gemm_kernel<kBwd>, mA, mP, mA2, mB2, ga);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  return launch_status();
+}
+
 // out16 = bf16(s . A.B) (and out16b if given) for a rank-r down projection: A is t x K
 // (K-major), B given by its map (ncols = r). One launch; with split-K the partial sums meet
 // in ws.acc32 and the last CTA of each 128-token tile rounds them.
@@ -603,7 +634,7 @@ int qlora_linear_fwd(const uint16_t* X, int64_t t, const nf4_weight* W, const ui
   // Y = X . W' + sT . L2
   CUtensorMap mA, mP, mA2, mB2;
   if (!map_bf16(&mA, X, h, t, 64, 128) ||
-      !make_map_2d(&mP, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, h / 2, o, h / 2, 32, 256, false) ||
+      !make_map_2d(&mP, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, h / 2, o, h / 2, 32, tc::BNH, false) ||
       !map_bf16(&mA2, sT, r, t, 64, 128) || !map_bf16(&mB2, L2, o, r, 64, 64))
     return QLORA_ERR_CUDA;
   Nf4GemmArgs ga{};
@@ -616,13 +647,7 @@ int qlora_linear_fwd(const uint16_t* X, int64_t t, const nf4_weight* W, const ui
   ga.num_lkb = static_cast<int>((r + 63) / 64);
   ga.out = Y;
   ga.tab = device_table();
-  dim3 grid(static_cast<unsigned>((o + 255) / 256), static_cast<unsigned>((t + tc::BM - 1) / tc::BM));
-  {
-    prof::Scope ps(prof::kGemmFwd, st);
-    nf4_gemm_kernel<false><<<grid, tc::kThreads, tc::nf4_gemm_smem_bytes(), st>>>(mA, mP, mA2,
-                                                                                mB2, ga);
-  }
-  return launch_status();
+  return launch_nf4_gemm<false>(mA, mP, mA2, mB2, ga, t, o, st, prof::kGemmFwd);
 }
 
 int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t t, const nf4_weight* W,
@@ -669,7 +694,7 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t t, const nf4
     CUtensorMap mA, mP, mA2, mB2;
     if (!map_bf16(&mA, dY, o, t, 64, 128) ||
         !make_map_2d(&mP, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, h / 2, o, h / 2, 32, 64, false) ||
-        !map_bf16(&mA2, sU, r, t, 64, 128) || !map_bf16(&mB2, L1, r, h, 64, 256))
+        !map_bf16(&mA2, sU, r, t, 64, 128) || !map_bf16(&mB2, L1, r, h, 64, tc::BNH))
       return QLORA_ERR_CUDA;
     Nf4GemmArgs ga{};
     ga.q8 = W->absmax_q8;
@@ -681,13 +706,7 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t t, const nf4
     ga.num_lkb = static_cast<int>((r + 63) / 64);
     ga.out = dX;
     ga.tab = device_table();
-    dim3 grid(static_cast<unsigned>((h + 255) / 256), static_cast<unsigned>((t + tc::BM - 1) / tc::BM));
-    {
-      prof::Scope ps(prof::kGemmBwd, st);
-      nf4_gemm_kernel<true><<<grid, tc::kThreads, tc::nf4_gemm_smem_bytes(), st>>>(mA, mP, mA2,
-                                                                                 mB2, ga);
-    }
-    if ((rc = launch_status())) return rc;
+    if ((rc = launch_nf4_gemm<true>(mA, mP, mA2, mB2, ga, t, h, st, prof::kGemmBwd))) return rc;
   }
 
   // dL1 = X^T . sU (h x r) and dL2^T = dY^T . sT (o x r), reductions over the t tokens
