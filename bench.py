@@ -174,6 +174,9 @@ def step_all(layers, world):
         dp.allreduce_adapter_grads([g for L in layers for g in (L.dL1, L.dL2)])
 
 
+QUEUE_SLEEP_CYCLES = 40_000_000   # ~20 ms at 1.965 GHz: time for the host to queue a loop
+
+
 def timed(fn, steps, warmup, world, dev):
     """Device time of `steps` calls of fn (after `warmup`), max over ranks, in ms."""
     from bit_quantized_lora_03_b200 import dp
@@ -239,8 +242,20 @@ def gemv_leg(dev, peaks, l2_bytes):
                 it[0] += 1
                 B.qlora_linear_fwd(X, q, L1, L2, 2.0, Y=Y, want_sT=False, ws=ws)
             reps = 4 * ncopy
-            ms = timed(call, reps, ncopy, 1, dev) / reps
+            host_ms = timed(call, reps, ncopy, 1, dev) / reps
+            # queued behind a device-side sleep, so that the events time the GPU work of
+            # back-to-back calls rather than the host's launch rate
+            torch.cuda.synchronize()
+            torch.cuda._sleep(QUEUE_SLEEP_CYCLES)
+            start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            start.record()
+            for _ in range(reps):
+                call()
+            end.record()
+            torch.cuda.synchronize()
+            ms = start.elapsed_time(end) / reps
             with B.KernelProfile() as prof:
+                torch.cuda._sleep(QUEUE_SLEEP_CYCLES)
                 for _ in range(reps):
                     call()
             k_ms = prof.ms["nf4_gemv_kernel"] / max(1, prof.launches["nf4_gemv_kernel"])
@@ -249,6 +264,7 @@ def gemv_leg(dev, peaks, l2_bytes):
             out.append({
                 "weight": name, "t": t, "packed_bytes": packed,
                 "call_us": round(ms * 1e3, 2),
+                "host_bound_call_us": round(host_ms * 1e3, 2),
                 "call_packed_gbs": round(packed / (ms * 1e-3) / 1e9, 1),
                 "gemv_kernel_us": round(k_ms * 1e3, 2),
                 "gemv_kernel_packed_gbs": round(packed / (k_ms * 1e-3) / 1e9, 1),

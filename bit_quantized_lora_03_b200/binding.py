@@ -27,6 +27,7 @@ QLORA_ERR_SCRATCH_LIMIT = -7
 QLORA_STATIC_SCRATCH_BYTES = 8 << 20
 QLORA_DEV_NONFINITE = 1
 QLORA_DEV_TIMEOUT = 2
+QLORA_DEV_LAUNCH = 4
 
 # Every symbol the header declares, with its ctypes signature.
 _PTR = ctypes.c_void_p
@@ -43,6 +44,7 @@ SIGNATURES = {
     "qlora_bwd_workspace_bytes": (ctypes.c_size_t, [_I64, _I64, _I64, _I64]),
     "qlora_get_last_status": (ctypes.c_int, [_PTR]),
     "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "qlora_set_gemv_max_ctas": (ctypes.c_int, [ctypes.c_int]),
     "qlora_profile_begin": (ctypes.c_int, [ctypes.c_int]),
     "qlora_profile_end": (ctypes.c_int, [_PTR, _PTR, ctypes.c_int]),
     "qlora_kernel_name": (ctypes.c_char_p, [ctypes.c_int]),
@@ -263,6 +265,11 @@ class KernelProfile:
             self.ms[name] = ms[k]
             self.launches[name] = n[k]
         return False
+
+
+def set_gemv_max_ctas(n: int) -> int:
+    """Cap the decode GEMV's CTA count (n <= 0: one per SM); returns the previous cap."""
+    return int(lib().qlora_set_gemv_max_ctas(int(n)))
 
 
 def last_status(stream=None) -> int:

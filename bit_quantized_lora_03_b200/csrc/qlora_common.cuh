@@ -16,6 +16,7 @@ __device__ unsigned int g_status;
 
 constexpr unsigned kDevNonfinite = 1u;
 constexpr unsigned kDevTimeout = 2u;
+constexpr unsigned kDevLaunch = 4u;
 
 // A bounded wait gives up after this long (nanoseconds of the global timer). Every legitimate
 // wait inside one CTA is shorter than a millisecond at the sizes this library accepts.

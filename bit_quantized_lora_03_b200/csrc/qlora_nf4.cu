@@ -23,6 +23,8 @@ using namespace qlora;
 
 namespace {
 
+std::atomic<int> g_gemv_max_ctas{0};  // cap on the decode GEMV's CTAs (0 = one per SM)
+
 // ------------------------------------------------------------------------------------------
 // NF4 codebook ("QLoRA in LLMs" section 5; "Idea one: NF4" on goodomens.studio; "Key
 // Components" on docs.skillversehub.com): 16 levels at standard-normal quantiles, an exact
@@ -121,6 +123,10 @@ int current_device(int* dev_out) {
                                  static_cast<int>(tc::nf4_gemm_smem_bytes())) == cudaSuccess;
     fine &= cudaFuncSetAttribute(nf4_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(tc::nf4_gemm_smem_bytes())) == cudaSuccess;
+    fine &= cudaFuncSetAttribute(nf4_gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(gv::smem_bytes())) == cudaSuccess;
+    fine &= cudaFuncSetAttribute(nf4_gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(gv::smem_bytes())) == cudaSuccess;
     fine &= cudaFuncSetAttribute(tc_gemm_kernel<false, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tcg::kMaxSmem) == cudaSuccess;
@@ -429,6 +435,10 @@ int qlora_nf4_codebook(float* levels, float* midpoints) {
   return QLORA_OK;
 }
 
+int qlora_set_gemv_max_ctas(int n) {
+  return g_gemv_max_ctas.exchange(n > 0 ? n : 0);
+}
+
 const char* qlora_status_string(int status) {
   switch (status) {
     case QLORA_OK: return "QLORA_OK";
@@ -603,20 +613,23 @@ int qlora_linear_fwd(const uint16_t* X, int64_t t, const nf4_weight* W, const ui
     ga.o = o;
     ga.t = static_cast<int>(t);
     ga.tab = device_table();
-    const int64_t nblk = h / 64;
-    const int64_t row_ctas = (o + 255) / 256;
-    // enough K slices for ~4 CTAs (16 warps) per SM
-    int64_t splits = std::max<int64_t>(1, (int64_t(sms) * 4 + row_ctas - 1) / row_ctas);
-    splits = std::min(splits, nblk);
-    ga.blocks_per_split = static_cast<int>((nblk + splits - 1) / splits);
-    const int64_t ysplits = (nblk + ga.blocks_per_split - 1) / ga.blocks_per_split;
-    dim3 grid(static_cast<unsigned>(row_ctas), static_cast<unsigned>(ysplits));
+    // one CTA of 16 warps per SM (fewer when there are fewer units than warps, or capped)
+    const int64_t units = (o / gv::kTileRows) * ((h / 64 + 1) / 2);
+    int64_t ctas = std::min<int64_t>(sms, (units + gv::kWarps - 1) / gv::kWarps);
+    const int cap = g_gemv_max_ctas.load(std::memory_order_relaxed);
+    if (cap > 0) ctas = std::min<int64_t>(ctas, cap);
+    dim3 grid(static_cast<unsigned>(ctas));
+    // codes as 32-row x 64-byte boxes (one unit each)
+    CUtensorMap mC;
+    if (!make_map_2d(&mC, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, h / 2, o, h / 2, 64,
+                     gv::kTileRows, false))
+      return QLORA_ERR_CUDA;
     {
       prof::Scope ps(prof::kGemv, st);
       if (t <= 8)
-        nf4_gemv_kernel<1><<<grid, 128, 0, st>>>(ga);
+        nf4_gemv_kernel<1><<<grid, gv::kThreads, gv::smem_bytes(), st>>>(ga, mC);
       else
-        nf4_gemv_kernel<2><<<grid, 128, 0, st>>>(ga);
+        nf4_gemv_kernel<2><<<grid, gv::kThreads, gv::smem_bytes(), st>>>(ga, mC);
     }
     if ((rc = launch_status())) return rc;
     dim3 fgrid(static_cast<unsigned>((o + 255) / 256), static_cast<unsigned>(t));

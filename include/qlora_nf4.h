@@ -75,8 +75,10 @@ enum {
 /* Device-side fault bits (positive), OR-ed into the status word by the kernels. */
 enum {
   QLORA_DEV_NONFINITE = 1,          /* nf4_quantize met a NaN or infinite weight             */
-  QLORA_DEV_TIMEOUT = 2             /* a kernel's bounded internal wait expired; outputs of
+  QLORA_DEV_TIMEOUT = 2,            /* a kernel's bounded internal wait expired; outputs of
                                        that call are unspecified                              */
+  QLORA_DEV_LAUNCH = 4              /* a kernel found its launch unusable (e.g. too little
+                                       shared memory) and did no work                         */
 };
 
 /* A packed NF4 weight: caller-owned device buffers plus the logical shape.
@@ -195,6 +197,14 @@ QLORA_API int qlora_get_last_status(qlora_stream_t stream);
 QLORA_API int qlora_profile_begin(int capacity);
 QLORA_API int qlora_profile_end(double *ms, int64_t *launches, int nkinds);
 QLORA_API const char *qlora_kernel_name(int kind);
+
+/* Launch shape of the decode GEMV (t <= 16), a scheduling knob with no counterpart in the
+ * method. By default the GEMV runs one CTA of 16 warps per SM and splits its units (32 rows x
+ * 128 inputs) evenly over all their warps. qlora_set_gemv_max_ctas(n) caps that CTA count at
+ * n for later calls on every device (n <= 0 restores the default), e.g. to leave SMs to work
+ * on another stream; results do not depend on it beyond fp32 summation order. Returns the
+ * previous cap (0 = none). Process-wide; not ordered with calls in flight on other threads. */
+QLORA_API int qlora_set_gemv_max_ctas(int n);
 
 /* A static, human-readable name for any QLORA_* code (never NULL). */
 QLORA_API const char *qlora_status_string(int status);

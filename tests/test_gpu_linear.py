@@ -127,3 +127,15 @@ def test_training_shape_linear_sampled():
     _, dL1_ref, dL2_ref, _ = O.qlora_linear_bwd(dY, X, Wdq, L1, L2, li.s)
     assert_close_rms(f32(dL1), dL1_ref, "dL1")
     assert_close_rms(f32(dL2), dL2_ref, "dL2")
+
+
+@pytest.mark.parametrize("t,ctas", [(1, 1), (5, 3), (12, 1), (16, 2)])
+def test_decode_gemv_long_warp_runs(t, ctas):
+    """Few CTAs give every warp a long run of units: it crosses row tiles and scale segments
+    (h = 64 x 67: 34 units per row, more than one 32-unit segment, the last unit one block)."""
+    li = inputs.random_linear(t, 64 * 67, 576, 16, 1.5, seed=500 + t, with_grad=False)
+    prev = B.set_gemv_max_ctas(ctas)
+    try:
+        _check_fwd(li)
+    finally:
+        B.set_gemv_max_ctas(prev)
