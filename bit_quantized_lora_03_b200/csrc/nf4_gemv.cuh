@@ -21,9 +21,11 @@
 // 64 bytes) per unit into a three-slot ring of shared memory, so a whole SM has ~96 KB of HBM
 // reads outstanding without spending registers on them. The 8-bit block scales of its rows
 // arrive in segments of up to 16 units, copied asynchronously one segment ahead; the
-// activations come through L1 one unit ahead (up to 8 tokens). When the run leaves a row tile,
-// and at its end, the warp adds its partial sums to a t x o fp32 buffer (one atomic per
-// output); a finalize kernel adds the LoRA term sT.L2 and rounds to bf16.
+// activations come through L1. When the run leaves a row tile, and at its end, the warp adds
+// its partial sums to a t x o fp32 buffer (one atomic per output) and the number of units it
+// did to the tile's counter; the warp that completes a tile adds the LoRA term sT.L2 to its
+// 32 rows and writes them in bf16. sT = bf16(s . X.L1) comes from gemv_lora_down_kernel, one
+// cluster of 8 CTAs launched just before, which also zeroes the fp32 buffer and the counters.
 #pragma once
 
 #include "nf4_codec.cuh"
@@ -64,8 +66,14 @@ constexpr int kSlotSeg = kDepth * kUnitBytes;
 constexpr int kSlotBars = kSlotSeg + 2 * kSegBytes;
 constexpr int kSlotBytes = (kSlotBars + kDepth * 8 + 127) / 128 * 128;
 // The table must start on a 64 KB boundary of the shared window; warp slots fill the space
-// before it and after it. Whatever the window's base, 64 KB + (warps + 1) slots are enough.
-constexpr size_t smem_bytes() { return kTableBytes + (kWarps + 1) * static_cast<size_t>(kSlotBytes); }
+// before it and after it. Whatever the window's base, 64 KB + (warps + 1) slots are enough;
+// sT (bf16, up to 16 tokens x rank 256) follows them.
+constexpr int kMaxTokens = 16;
+constexpr int kMaxRank = 256;
+constexpr int kDownParts = 8;  // partial sums written by the LoRA-down kernel (one per cluster)
+constexpr int kSTBytes = kMaxTokens * kMaxRank * 2;
+constexpr size_t slots_end() { return kTableBytes + (kWarps + 1) * static_cast<size_t>(kSlotBytes); }
+constexpr size_t smem_bytes() { return slots_end() + kSTBytes; }
 static_assert(kSegWords * 4 >= 2 * kSegUnits + 6, "a row segment plus its alignment fits");
 static_assert(smem_bytes() <= 232448 - 1024, "fits the opt-in shared memory of one CTA");
 }  // namespace gv
@@ -74,11 +82,18 @@ struct GemvArgs {
   const uint8_t* codes;
   const uint8_t* q8;
   const float* s2;
-  const uint16_t* X;  // t x h bf16
-  float* Y32;         // t x o fp32, zeroed by the caller
+  const uint16_t* X;   // t x h bf16
+  const float* Tpart;  // gd::kClusters partial sums of X.L1, each t x r fp32
+  uint16_t* sT_out;    // t x r bf16 s . X.L1 for the caller (may be null)
+  float s;
+  const uint16_t* L2;  // r x o bf16
+  uint16_t* Y;         // t x o bf16 (output)
+  float* Y32;          // t x o fp32, zero on entry
+  unsigned* tile_cnt;  // o / 32 unit counters, zero on entry
   int64_t h;
   int64_t o;
   int t;
+  int r;
   Nf4Table tab;
 };
 
@@ -264,6 +279,34 @@ __device__ __forceinline__ void gemv_flush(float (&acc)[2][NT][4], const GemvArg
       }
 }
 
+// The last warp to add to a row tile finishes it: Y[n][row] = bf16(Y32[n][row] + sum_c
+// sT[n][c] L2[c][row]) for its 32 rows, lane = row. The fp32 sums of the other warps are read
+// from L2 after the counter showed them all done (each adder fenced before counting).
+template <int NT>
+__device__ __forceinline__ void gemv_finish_tile(const GemvArgs& a, const uint16_t* sts,
+                                                 int64_t tile, int lane) {
+  const int64_t row = tile * gv::kTileRows + lane;
+  float y[NT * 8];
+#pragma unroll
+  for (int n = 0; n < NT * 8; ++n)
+    y[n] = n < a.t ? __ldcg(a.Y32 + static_cast<int64_t>(n) * a.o + row) : 0.f;
+  for (int c0 = 0; c0 < a.r; c0 += 8) {  // r % 16 == 0: eight loads in flight per lane
+    float l2[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      l2[j] = bf16_bits_to_float(__ldg(a.L2 + static_cast<int64_t>(c0 + j) * a.o + row));
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int n = 0; n < NT * 8; ++n)
+        if (n < a.t) y[n] = fmaf(bf16_bits_to_float(sts[n * gv::kMaxRank + c0 + j]), l2[j], y[n]);
+  }
+#pragma unroll
+  for (int n = 0; n < NT * 8; ++n)
+    if (n < a.t)
+      a.Y[static_cast<int64_t>(n) * a.o + row] = __bfloat16_as_ushort(__float2bfloat16_rn(y[n]));
+}
+
 template <int NT>  // NT: n8 token tiles (1 for t <= 8, 2 for t <= 16)
 __global__ void __launch_bounds__(gv::kThreads, 1)
     nf4_gemv_kernel(const GemvArgs args, const __grid_constant__ CUtensorMap map_codes) {
@@ -284,11 +327,13 @@ __global__ void __launch_bounds__(gv::kThreads, 1)
   };
   const uint32_t slot = slot_of(static_cast<uint32_t>(warp));
   // the last warp's slot ends last; the test is the same in every thread of the CTA
-  if (slot_of(kWarps - 1) + kSlotBytes > sbase + dyn_bytes || tab + kTableBytes > sbase + dyn_bytes) {
+  if (sbase + slots_end() + kSTBytes > sbase + dyn_bytes || slot_of(kWarps - 1) + kSlotBytes > sbase + slots_end() ||
+      tab + kTableBytes > sbase + slots_end()) {
     if (threadIdx.x == 0) report(kDevLaunch);  // launched with too little shared memory
     return;
   }
   float2* table = reinterpret_cast<float2*>(smem + (tab - sbase));  // [256 byte values][32 lanes]
+  uint16_t* sts = reinterpret_cast<uint16_t*>(smem + slots_end());   // [token][kMaxRank]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (slot - sbase) + kSlotBars);
 
   const int64_t nblk = args.h / kBlock;
@@ -329,6 +374,17 @@ __global__ void __launch_bounds__(gv::kThreads, 1)
     const int e = i >> 5;
     table[i] = make_float2(args.tab.level[e >> 4], args.tab.level[e & 15]);
   }
+  // sT = bf16(s . X.L1) from the LoRA-down kernel's partial sums (launched just before this
+  // kernel, which may start early: wait for its completion and memory first)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  for (int i = threadIdx.x; i < args.t * args.r; i += kThreads) {
+    float v = 0.f;
+#pragma unroll
+    for (int p = 0; p < kDownParts; ++p) v += __ldcg(args.Tpart + p * args.t * args.r + i);
+    const uint16_t b = __bfloat16_as_ushort(__float2bfloat16_rn(args.s * v));
+    sts[(i / args.r) * kMaxRank + i % args.r] = b;
+    if (blockIdx.x == 0 && args.sT_out) args.sT_out[i] = b;
+  }
   __syncthreads();
   if (nrun <= 0) return;
 
@@ -342,6 +398,7 @@ __global__ void __launch_bounds__(gv::kThreads, 1)
       for (int i = 0; i < 4; ++i) acc[mt][nt][i] = 0.f;
 
   int cb = 0;
+  int tile_units = 0;  // units of the current row tile done by this warp
   int i = 0;        // position in the run
   int e = 0;        // its ring entry, i % kDepth
   uint32_t ph = 0;  // the entry's fill parity, (i / kDepth) & 1
@@ -408,7 +465,22 @@ __global__ void __launch_bounds__(gv::kThreads, 1)
           for (int j = 0; j < 4; ++j) xc[nt][j] = xn[nt][j];
       }
     }
-    if (nxt.u0 == nxt.u1 || nxt.tile != cur.tile) gemv_flush<NT>(acc, args, cur.tile, g, q);
+    tile_units += cur.u1 - cur.u0;
+    if (nxt.u0 == nxt.u1 || nxt.tile != cur.tile) {
+      // add the tile's sums, then count its units; the warp that completes the tile
+      // finishes it (the fence makes this warp's sums visible before its count)
+      gemv_flush<NT>(acc, args, cur.tile, g, q);
+      __threadfence();
+      __syncwarp();
+      unsigned before_me = 0;
+      if (lane == 0) before_me = atomicAdd(args.tile_cnt + cur.tile, static_cast<unsigned>(tile_units));
+      before_me = __shfl_sync(0xffffffffu, before_me, 0);
+      if (before_me + tile_units == upt) {
+        __threadfence();
+        gemv_finish_tile<NT>(args, sts, cur.tile, lane);
+      }
+      tile_units = 0;
+    }
     if (nxt.u0 == nxt.u1) break;
     // move to the next segment; its buffer's copies were issued one segment ago
     cur = nxt;
@@ -422,22 +494,112 @@ __global__ void __launch_bounds__(gv::kThreads, 1)
   }
 }
 
-// Y[n][j] = bf16( Y32[n][j] + sum_c sT[n][c] * L2[c][j] ) with sT = bf16(s . X.L1): the LoRA
-// up-projection folded into the GEMV's output conversion. Grid (ceil(o/256), t).
-__global__ void __launch_bounds__(256) gemv_lora_finalize_kernel(
-    const float* __restrict__ Y32, const uint16_t* __restrict__ sT, const uint16_t* __restrict__ L2,
-    uint16_t* __restrict__ Y, int64_t o, int r) {
-  __shared__ float sTs[256];
-  const int n = blockIdx.y;
-  for (int c = threadIdx.x; c < r; c += blockDim.x)
-    sTs[c] = bf16_bits_to_float(sT[static_cast<int64_t>(n) * r + c]);
+// T = X.L1 for the decode path (t <= 16) as partial sums: 8 clusters of 8 CTAs; CTA q of
+// cluster p sums its share of the inputs k into an fp32 t x r partial in shared memory (thread
+// = column pair x a stride of k, four rows in flight), and the cluster's CTA 0 adds its eight
+// CTAs' partials over distributed shared memory and writes partial p. The GEMV adds the 8
+// partials, scales by s and rounds once to bf16 (the tensor-core path's sT up to summation
+// order). The grid also zeroes the GEMV's fp32 output sums and tile counters.
+namespace gd {
+constexpr int kClusterCtas = 8;
+constexpr int kClusters = gv::kDownParts;
+constexpr int kCtas = kClusterCtas * kClusters;
+constexpr int kThreads = 256;
+constexpr size_t smem_bytes(int t, int r) {
+  return (static_cast<size_t>(2 * kThreads) * t + static_cast<size_t>(t) * r) * 4;
+}
+}  // namespace gd
+
+__device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t rank) {
+  uint32_t raddr;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(raddr) : "r"(smem_addr(local)), "r"(rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(raddr) : "memory");
+  return v;
+}
+
+__global__ void __cluster_dims__(gd::kClusterCtas, 1, 1) __launch_bounds__(gd::kThreads)
+    gemv_lora_down_kernel(const uint16_t* __restrict__ X, const uint16_t* __restrict__ L1,
+                          float* Tpart, float* Y32, unsigned* tile_cnt, int64_t h, int64_t o,
+                          int t, int r) {
+  extern __shared__ __align__(16) float dsm[];
+  const int tid = threadIdx.x;
+  const uint32_t rank = cluster_ctarank();
+  const int cluster = blockIdx.x / gd::kClusterCtas;
+  // the GEMV launched after this kernel may be scheduled now (it waits for this grid's
+  // completion before reading anything written here)
+  asm volatile("griddepcontrol.launch_dependents;");
+
+  // zero the GEMV's accumulators (t x o floats, o / 32 counters)
+  {
+    const int64_t gt = static_cast<int64_t>(blockIdx.x) * gd::kThreads + tid;
+    const int64_t gn = static_cast<int64_t>(gd::kCtas) * gd::kThreads;
+    float4* y4 = reinterpret_cast<float4*>(Y32);
+    for (int64_t i = gt; i < static_cast<int64_t>(t) * o / 4; i += gn) y4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int64_t i = gt; i < o / 32; i += gn) tile_cnt[i] = 0u;
+  }
+
+  const int ncp = r / 2;                // column pairs
+  const int nkg = gd::kThreads / ncp;   // k strides (r <= 256, r % 16 == 0: exact)
+  const int cp = tid % ncp, kg = tid / ncp;
+  // this CTA's inputs: an even share of the 2-row pairs
+  const int64_t pairs = h / 2;
+  const int64_t p0 = pairs * blockIdx.x / gd::kCtas, p1 = pairs * (blockIdx.x + 1) / gd::kCtas;
+  float acc[16][2];
+#pragma unroll
+  for (int n = 0; n < 16; ++n) acc[n][0] = acc[n][1] = 0.f;
+  for (int64_t pb = p0 + kg; pb < p1; pb += 4 * nkg) {
+    uint32_t la[4], lb[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t pr = pb + u * nkg;
+      const int64_t k = 2 * (pr < p1 ? pr : p0);
+      la[u] = __ldg(reinterpret_cast<const uint32_t*>(L1 + k * r) + cp);
+      lb[u] = __ldg(reinterpret_cast<const uint32_t*>(L1 + (k + 1) * r) + cp);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t pr = pb + u * nkg;
+      if (pr >= p1) break;
+      const int64_t k = 2 * pr;
+      const float a0 = bf16_bits_to_float(la[u] & 0xffffu), a1 = bf16_bits_to_float(la[u] >> 16);
+      const float b0 = bf16_bits_to_float(lb[u] & 0xffffu), b1 = bf16_bits_to_float(lb[u] >> 16);
+#pragma unroll
+      for (int n = 0; n < 16; ++n) {
+        if (n < t) {
+          const uint32_t xv = __ldg(reinterpret_cast<const uint32_t*>(X + static_cast<int64_t>(n) * h + k));
+          const float x0 = bf16_bits_to_float(xv & 0xffffu), x1 = bf16_bits_to_float(xv >> 16);
+          acc[n][0] = fmaf(x1, b0, fmaf(x0, a0, acc[n][0]));
+          acc[n][1] = fmaf(x1, b1, fmaf(x0, a1, acc[n][1]));
+        }
+      }
+    }
+  }
+  // [kg][n][c] partials -> this CTA's t x r sums
+  float* red = dsm;
+  float* part = dsm + static_cast<size_t>(2 * gd::kThreads) * t;
+#pragma unroll
+  for (int n = 0; n < 16; ++n)
+    if (n < t) {
+      red[(kg * t + n) * r + 2 * cp] = acc[n][0];
+      red[(kg * t + n) * r + 2 * cp + 1] = acc[n][1];
+    }
   __syncthreads();
-  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (j >= o) return;
-  float y = Y32[static_cast<int64_t>(n) * o + j];
-  for (int c = 0; c < r; ++c)
-    y = fmaf(sTs[c], bf16_bits_to_float(L2[static_cast<int64_t>(c) * o + j]), y);
-  Y[static_cast<int64_t>(n) * o + j] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+  for (int i = tid; i < t * r; i += gd::kThreads) {
+    float v = 0.f;
+    for (int j = 0; j < nkg; ++j) v += red[j * t * r + i];
+    part[i] = v;
+  }
+  cluster_sync();
+  if (rank == 0) {
+    for (int i = tid; i < t * r; i += gd::kThreads) {
+      float v = 0.f;
+#pragma unroll
+      for (uint32_t q = 0; q < gd::kClusterCtas; ++q) v += ld_dsmem_f32(part + i, q);
+      Tpart[static_cast<int64_t>(cluster) * t * r + i] = v;
+    }
+  }
+  cluster_sync();  // the partials stay in place until the cluster's CTA 0 has read them
 }
 
 }  // namespace qlora

@@ -123,6 +123,8 @@ int current_device(int* dev_out) {
                                  static_cast<int>(tc::nf4_gemm_smem_bytes())) == cudaSuccess;
     fine &= cudaFuncSetAttribute(nf4_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(tc::nf4_gemm_smem_bytes())) == cudaSuccess;
+    fine &= cudaFuncSetAttribute(gemv_lora_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(gd::smem_bytes(16, 256))) == cudaSuccess;
     fine &= cudaFuncSetAttribute(nf4_gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(gv::smem_bytes())) == cudaSuccess;
     fine &= cudaFuncSetAttribute(nf4_gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -156,11 +158,11 @@ int launch_status() {
 // ------------------------------------------------------------------------------------------
 namespace prof {
 enum Kind {
-  kQuant = 0, kDequant, kGemv, kGemvFinalize, kTcGemm, kGemmFwd, kGemmBwd, kKinds
+  kQuant = 0, kDequant, kGemv, kGemvLoraDown, kTcGemm, kGemmFwd, kGemmBwd, kKinds
 };
 const char* const kNames[kKinds] = {
     "nf4_quantize_kernel", "nf4_dequantize_kernel", "nf4_gemv_kernel",
-    "gemv_lora_finalize_kernel", "tc_gemm_kernel",
+    "gemv_lora_down_kernel", "tc_gemm_kernel",
     "nf4_gemm_kernel<fwd>", "nf4_gemm_kernel<bwd>"};
 static_assert(kKinds == QLORA_KERNEL_KINDS, "kernel kinds");
 
@@ -281,9 +283,26 @@ size_t lora_region_bytes(int64_t t, int64_t r) {
   return lora_acc_bytes(t, r) + lora_counter_bytes(t) + align256(static_cast<size_t>(t) * r * 2);
 }
 
-// fp32 t x o accumulator for the GEMV's split-K partial sums
-size_t gemv_region_bytes(int64_t t, int64_t o) {
-  return align256(static_cast<size_t>(t) * o * 4);
+// decode path (t <= 16): partial sums of X.L1 (gv::kDownParts x t x r fp32), the GEMV's fp32
+// t x o sums, its o / 32 tile counters
+struct GemvWs {
+  float* Tpart;
+  float* Y32;
+  unsigned* cnt;
+};
+size_t gemv_ws_bytes(int64_t t, int64_t o, int64_t r) {
+  return align256(static_cast<size_t>(gv::kDownParts) * t * r * 4) +
+         align256(static_cast<size_t>(t) * o * 4) + align256(static_cast<size_t>(o / 32) * 4);
+}
+GemvWs carve_gemv(void* base, int64_t t, int64_t o, int64_t r) {
+  uint8_t* b = reinterpret_cast<uint8_t*>(base);
+  GemvWs w;
+  w.Tpart = reinterpret_cast<float*>(b);
+  b += align256(static_cast<size_t>(gv::kDownParts) * t * r * 4);
+  w.Y32 = reinterpret_cast<float*>(b);
+  b += align256(static_cast<size_t>(t) * o * 4);
+  w.cnt = reinterpret_cast<unsigned*>(b);
+  return w;
 }
 
 constexpr int64_t kGemvMaxTokens = 16;
@@ -460,9 +479,8 @@ const char* qlora_status_string(int status) {
 
 size_t qlora_fwd_workspace_bytes(int64_t t, int64_t h, int64_t o, int64_t r) {
   if (check_linear_shape(t, h, o, r) != QLORA_OK) return 0;
-  size_t b = lora_region_bytes(t, r);
-  if (t <= kGemvMaxTokens) b += gemv_region_bytes(t, o);
-  return b;
+  if (t <= kGemvMaxTokens) return gemv_ws_bytes(t, o, r);
+  return lora_region_bytes(t, r);
 }
 
 size_t qlora_bwd_workspace_bytes(int64_t t, int64_t h, int64_t o, int64_t r) {
@@ -591,27 +609,32 @@ int qlora_linear_fwd(const uint16_t* X, int64_t t, const nf4_weight* W, const ui
   if ((rc = current_device(&dev))) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int sms = sm_count(dev);
-  LoraWs ws = carve_lora(workspace, t, r);
-
-  // T = X . L1 (t x r), then sT = bf16(s . T)
-  CUtensorMap mX, mL1;
-  if (!map_bf16(&mX, X, h, t, 64, 128) || !map_bf16(&mL1, L1, r, h, 64, 64)) return QLORA_ERR_CUDA;
-
   if (t <= kGemvMaxTokens) {
-    float* Y32 = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) +
-                                          lora_region_bytes(t, r));
-    if (cudaMemsetAsync(Y32, 0, static_cast<size_t>(t) * o * 4, st) != cudaSuccess)
-      return QLORA_ERR_CUDA;
-    if ((rc = lora_down<true>(mX, mL1, t, h, r, s, ws, ws.b16, sT_out, sms, st))) return rc;
+    // partial sums of X.L1 (+ zeroed sums and counters), then the GEMV, which forms
+    // sT = bf16(s . X.L1) and finishes Y
+    GemvWs gw = carve_gemv(workspace, t, o, r);
+    {
+      prof::Scope ps(prof::kGemvLoraDown, st);
+      gemv_lora_down_kernel<<<gd::kCtas, gd::kThreads, gd::smem_bytes(static_cast<int>(t), static_cast<int>(r)), st>>>(
+          X, L1, gw.Tpart, gw.Y32, gw.cnt, h, o, static_cast<int>(t), static_cast<int>(r));
+    }
+    if ((rc = launch_status())) return rc;
     GemvArgs ga{};
     ga.codes = W->codes;
     ga.q8 = W->absmax_q8;
     ga.s2 = W->absmax_s2;
     ga.X = X;
-    ga.Y32 = Y32;
+    ga.Tpart = gw.Tpart;
+    ga.sT_out = sT_out;
+    ga.s = s;
+    ga.L2 = L2;
+    ga.Y = Y;
+    ga.Y32 = gw.Y32;
+    ga.tile_cnt = gw.cnt;
     ga.h = h;
     ga.o = o;
     ga.t = static_cast<int>(t);
+    ga.r = static_cast<int>(r);
     ga.tab = device_table();
     // one CTA of 16 warps per SM (fewer when there are fewer units than warps, or capped)
     const int64_t units = (o / gv::kTileRows) * ((h / 64 + 1) / 2);
@@ -625,21 +648,32 @@ int qlora_linear_fwd(const uint16_t* X, int64_t t, const nf4_weight* W, const ui
                      gv::kTileRows, false))
       return QLORA_ERR_CUDA;
     {
+      // programmatic dependent launch: the GEMV's CTAs may start (table, first code loads)
+      // while the LoRA-down kernel runs; they wait for its results before using them
       prof::Scope ps(prof::kGemv, st);
-      if (t <= 8)
-        nf4_gemv_kernel<1><<<grid, gv::kThreads, gv::smem_bytes(), st>>>(ga, mC);
-      else
-        nf4_gemv_kernel<2><<<grid, gv::kThreads, gv::smem_bytes(), st>>>(ga, mC);
-    }
-    if ((rc = launch_status())) return rc;
-    dim3 fgrid(static_cast<unsigned>((o + 255) / 256), static_cast<unsigned>(t));
-    {
-      prof::Scope ps(prof::kGemvFinalize, st);
-      gemv_lora_finalize_kernel<<<fgrid, 256, 0, st>>>(Y32, ws.b16, L2, Y, o,
-                                                       static_cast<int>(r));
+      cudaLaunchConfig_t cfg{};
+      cfg.gridDim = grid;
+      cfg.blockDim = dim3(gv::kThreads);
+      cfg.dynamicSmemBytes = gv::smem_bytes();
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      const cudaError_t e = t <= 8 ? cudaLaunchKernelEx(&cfg, nf4_gemv_kernel<1>, ga, mC)
+                                   : cudaLaunchKernelEx(&cfg, nf4_gemv_kernel<2>, ga, mC);
+      if (e != cudaSuccess) return QLORA_ERR_CUDA;
     }
     return launch_status();
   }
+
+  LoraWs ws = carve_lora(workspace, t, r);
+
+  // T = X . L1 (t x r), then sT = bf16(s . T)
+  CUtensorMap mX, mL1;
+  if (!map_bf16(&mX, X, h, t, 64, 128) || !map_bf16(&mL1, L1, r, h, 64, 64)) return QLORA_ERR_CUDA;
+
 
   uint16_t* sT = ws.b16;
   if ((rc = lora_down<true>(mX, mL1, t, h, r, s, ws, sT, sT_out, sms, st))) return rc;
