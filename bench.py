@@ -54,13 +54,17 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+# the sources the fused NF4 GEMM is compiled from (its DRAM counters stay valid while these
+# files are unchanged)
+GEMM_SOURCES = ("nf4_gemm.cuh", "nf4_codec.cuh", "qlora_common.cuh")
+
+
 def kernel_source_hash() -> str:
     csrc = os.path.join(ROOT, "bit_quantized_lora_03_b200", "csrc")
     h = hashlib.sha256()
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for name in GEMM_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
