@@ -313,6 +313,35 @@ def codec_leg(dev, peaks):
     return res
 
 
+def stack65b_leg(dev, peaks, steps: int = 2, warmup: int = 1):
+    """The 65B-shaped stack (80 layers x 7 linears, 33.4 GB packed, t = 2048, r = 64): device
+    time of full fwd+bwd steps through all 560 linears."""
+    from bit_quantized_lora_03_b200 import binding as B
+    from bit_quantized_lora_03_b200.stack65b import Stack65B
+    import time as _time
+    t0 = _time.time()
+    st = Stack65B(dev)
+    setup_s = _time.time() - t0
+    ms = timed(st.step, steps, warmup, 1, dev)
+    status = B.last_status()
+    flops = st.flops_per_step()
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    res = {
+        "workload": "llama65b_stack_80x7_linears_fwd_bwd_t2048_r64",
+        "tokens_per_s": round(st.t * steps / (ms * 1e-3), 1),
+        "ms_per_step": round(ms / steps, 2), "steps": steps, "warmup": warmup,
+        "packed_weight_bytes": st.packed_bytes,
+        "tflop_per_step": round(flops / 1e12, 2),
+        "tflops": round(flops * steps / (ms * 1e-3) / 1e12, 1),
+        "frac_of_sustained_bf16": round(flops * steps / (ms * 1e-3) / 1e12 / peak, 4),
+        "launches_per_step": 6 * len(st.lin),
+        "setup_s": round(setup_s, 1), "device_status": status,
+    }
+    del st
+    torch.cuda.empty_cache()
+    return res
+
+
 # ------------------------------------------------------------------------------------------
 # CPU oracle baseline (bounded sample)
 # ------------------------------------------------------------------------------------------
@@ -486,6 +515,7 @@ def main():
         torch.cuda.empty_cache()
         legs["decode_gemv"] = gemv_leg(dev, peaks, l2_bytes)
         legs["codec_llama7b_layer"] = codec_leg(dev, peaks)
+        legs["stack65b"] = stack65b_leg(dev, peaks)
         tps, sec, _ = oracle_sample(args.cpu_sample_tokens)
         cpu = {"value": round(tps, 3), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                "sample": (f"fwd+bwd of {args.cpu_sample_tokens} of the 4096 tokens, one linear per "

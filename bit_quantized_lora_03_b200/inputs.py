@@ -163,3 +163,50 @@ def random_linear(t: int, h: int, o: int, r: int, s: float, seed: int,
     L2 = normal_bf16((r, o), ADAPTER_SIGMA, g)
     dY = normal_bf16((t, o), 1.0, g) if with_grad else None
     return LinearInputs(f"random_t{t}_h{h}_o{o}_r{r}", Wt, X, L1, L2, s, dY)
+
+
+# ------------------------------------------------------------------------------------------
+# The 65B-shaped stack: 80 layers x the 7 linears of LLAMA65B_LINEARS, 2048 tokens, r = 64,
+# s = 0.25. Its 64.76 G weights are drawn on the device (a CPU draw of that size is too slow):
+# torch's CUDA generator, seeded 500 + 7 layer + i for the weight of linear i of a layer and
+# 100000 + 7 layer + i for its adapters (L1 then L2), N(0,0.02) and N(0,0.01) as elsewhere.
+# Every layer's linears read shared seeded inputs and upstream gradients (CPU generator):
+# X (t x 8192) seed 510 for the six linears with 8192 inputs, X (t x 22016) seed 511 for
+# down_proj; dY (t x 8192) seed 520 for the outputs of width 8192, dY (t x 22016) seed 521.
+# ------------------------------------------------------------------------------------------
+STACK65B_LAYERS = 80
+STACK65B_TOKENS = 2048
+STACK65B_RANK = 64
+STACK65B_S = 0.25
+
+
+def _device_gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+def stack65b_weight(layer: int, i: int, device) -> torch.Tensor:
+    """Wt (o x h fp32, on `device`) of linear i of `layer`: N(0, 0.02), seed 500 + 7 layer + i."""
+    _, h, o = LLAMA65B_LINEARS[i]
+    g = _device_gen(500 + 7 * layer + i, device)
+    return torch.randn(o, h, generator=g, dtype=torch.float32, device=device) * torch.tensor(
+        W_SIGMA, dtype=torch.float32, device=device)
+
+
+def stack65b_adapters(layer: int, i: int, device, r: int = STACK65B_RANK):
+    """(L1 h x r, L2 r x o) bf16 on `device`: N(0, 0.01), seed 100000 + 7 layer + i."""
+    _, h, o = LLAMA65B_LINEARS[i]
+    g = _device_gen(100000 + 7 * layer + i, device)
+    sig = torch.tensor(ADAPTER_SIGMA, dtype=torch.float32, device=device)
+    L1 = (torch.randn(h, r, generator=g, dtype=torch.float32, device=device) * sig).to(torch.bfloat16)
+    L2 = (torch.randn(r, o, generator=g, dtype=torch.float32, device=device) * sig).to(torch.bfloat16)
+    return L1, L2
+
+
+def stack65b_activations(t: int = STACK65B_TOKENS):
+    """Shared inputs and upstream gradients: {8192: X, 22016: X} and {8192: dY, 22016: dY},
+    bf16 N(0,1) on the CPU."""
+    X = {8192: normal_bf16((t, 8192), 1.0, _gen(510)), 22016: normal_bf16((t, 22016), 1.0, _gen(511))}
+    dY = {8192: normal_bf16((t, 8192), 1.0, _gen(520)), 22016: normal_bf16((t, 22016), 1.0, _gen(521))}
+    return X, dY
