@@ -1,6 +1,7 @@
-// tcgen05 (5th-generation tensor core) GEMMs for the training-shape QLoRA linear on sm_100a.
+// tcgen05 (5th-generation tensor core) fused NF4 GEMM for the training-shape QLoRA linear on
+// sm_100a.
 //
-// 1) nf4_gemm_kernel<BWD>: the frozen-base product with the NF4 dequantization fused into the
+// nf4_gemm_kernel<BWD>: the frozen-base product with the NF4 dequantization fused into the
 //    producer stage and the LoRA product folded into the same TMEM accumulator:
 //       forward  (BWD = false):  Y  = X  . W'   + sT . L2      (M = t, N = o, K = h)
 //       backward (BWD = true):   dX = dY . W'^T + sU . L1^T    (M = t, N = h, K = o)
@@ -16,9 +17,7 @@
 //    (A = sT or sU, B = L2 or L1, both by TMA) run first, then the h/64 (or o/64) weight
 //    K-steps. The same 8 warps then drain TMEM to bf16.
 //
-// 2) tc_gemm_kernel<A_MN, B_MN>: a plain TMA-fed tcgen05 GEMM (both operands by TMA, either
-//    major-ness) with split-K and fp32 atomic or bf16 output, for the rank-r products
-//    T = X.L1, U = dY.L2^T, dL1 = X^T.sU and dL2^T = dY^T.sT.
+// (tc_gemm.cuh holds the plain tcgen05 GEMM for the rank-r products.)
 //
 // Every wait is bounded (qlora::mbar_wait); on expiry the CTA reports QLORA_DEV_TIMEOUT,
 // stops issuing, waits for its own copies and MMAs in flight, frees TMEM and returns.
@@ -362,288 +361,6 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     tc_fence_after();
     tmem_dealloc2(tmem_base, kTmemCols);
   }
-}
-
-// ------------------------------------------------------------------------------------------
-// Plain TMA-fed tcgen05 GEMM for the rank-r products.
-// D (M x Ncols) = A (M x K) . B (K x Ncols), Ncols <= 256 (one N tile), split-K over
-// blockIdx.z. A_MN / B_MN select MN-major operands (the TMA boxes are 64 x 64 atoms then).
-// The pipeline depth is chosen by the host from the B tile size.
-// ------------------------------------------------------------------------------------------
-namespace tcg {
-constexpr int BM = 128, BK = 64, MAX_STAGES = 8;
-constexpr int A_BYTES = BM * BK * 2;        // 16 KB
-constexpr int kThreads = 6 * 32;            // warps 0-3 epilogue, 4 TMA, 5 MMA
-constexpr int kTmaWarp = 4, kMmaWarp = 5;
-constexpr int kMaxSmem = 232448 - 1024;     // opt-in maximum per CTA on sm_100, less static smem
-// B tile bytes for a given MMA N (BNp, multiple of 16) and major-ness
-__host__ __device__ constexpr int b_bytes(int BNp, bool b_mn) {
-  return b_mn ? ((BNp + 63) / 64) * 8192 : BNp * 128;
-}
-__host__ __device__ constexpr int stage_bytes(int BNp, bool b_mn) {
-  return A_BYTES + ((b_bytes(BNp, b_mn) + 1023) / 1024) * 1024;
-}
-constexpr size_t smem_bytes(int stages, int BNp, bool b_mn) {
-  return 1024 + static_cast<size_t>(stages) * stage_bytes(BNp, b_mn) + 256;
-}
-}  // namespace tcg
-
-enum TcOutMode : int {
-  kOutAtomicRowMajor = 0,   // out32[m * ld + n] += acc
-  kOutAtomicTransposed = 1, // out32[n * ld + m] += acc
-  kOutRoundBf16 = 2,        // out32 (m * Ncols + n) += acc; the last CTA of each M tile then
-                            // writes bf16(alpha * out32) to out16a (and out16b if set)
-};
-
-struct TcGemmArgs {
-  int M;
-  int Ncols;         // real number of output columns (<= BNp)
-  int BNp;           // MMA N: Ncols rounded up to a multiple of 16
-  int num_kb;        // ceil(K / 64)
-  int kb_per_split;
-  int splits;        // gridDim.z
-  int stages;
-  float alpha;
-  int out_mode;
-  float* out32;
-  int64_t ld;
-  uint16_t* out16a;
-  uint16_t* out16b;
-  unsigned* counters;  // kOutRoundBf16: one per M tile, zeroed by the caller
-};
-
-#ifdef QLORA_TRACE
-constexpr int kTraceCtas = 8192;
-__device__ unsigned long long g_trace[kTraceCtas][8];
-__device__ __forceinline__ void trace_stamp(int slot) {
-  const unsigned cta = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
-  if (cta < kTraceCtas) g_trace[cta][slot] = global_timer_ns();
-}
-#define QLORA_STAMP(i) trace_stamp(i)
-#else
-#define QLORA_STAMP(i)
-#endif
-
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
-}
-
-template <bool A_MN, bool B_MN>
-__global__ void __launch_bounds__(tcg::kThreads, 1)
-    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const TcGemmArgs args) {
-  using namespace tcg;
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ uint32_t last_flag;
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  const int BNp = args.BNp;
-  const int STAGES = args.stages;
-  const int SB = stage_bytes(BNp, B_MN);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * SB);
-  uint64_t* empty = full + MAX_STAGES;
-  uint64_t* acc_full = empty + MAX_STAGES;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
-  volatile uint32_t* abort_flag = tmem_holder + 1;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * BM;
-  const int kb0 = blockIdx.z * args.kb_per_split;
-  const int kb1 = min(args.num_kb, kb0 + args.kb_per_split);
-  const int nk = kb1 - kb0;
-  const uint32_t tmem_cols = BNp <= 32 ? 32u : (BNp <= 64 ? 64u : (BNp <= 128 ? 128u : 256u));
-  const int b_atoms = (BNp + 63) / 64;
-  const uint32_t bbytes = static_cast<uint32_t>(b_bytes(BNp, B_MN));
-
-  if (threadIdx.x == 0) {
-    QLORA_STAMP(0);
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    mbar_init(acc_full, 1);
-    *abort_flag = 0u;
-    fence_mbar_init();
-  }
-  if (warp == kMmaWarp) {
-    tmem_alloc(tmem_holder, tmem_cols);
-    tmem_relinquish();
-  }
-  if (warp == kTmaWarp && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_holder;
-  if (threadIdx.x == 0) QLORA_STAMP(1);
-
-  if (warp == kTmaWarp) {
-    if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < nk; ++i) {
-        const int slot = i % STAGES;
-        const uint32_t ph = (i / STAGES) & 1;
-        if (!mbar_wait(&empty[slot], ph ^ 1u, abort_flag)) break;
-        const int kb = kb0 + i;
-        mbar_arrive_expect_tx(&full[slot], A_BYTES + bbytes);
-        uint8_t* a_dst = smem + slot * SB;
-        if (!A_MN) {
-          tma_load_2d(a_dst, &tmA, &full[slot], kb * BK, m0);
-        } else {
-          tma_load_2d(a_dst, &tmA, &full[slot], m0, kb * BK);
-          tma_load_2d(a_dst + 8192, &tmA, &full[slot], m0 + 64, kb * BK);
-        }
-        uint8_t* b_dst = a_dst + A_BYTES;
-        if (!B_MN) {
-          tma_load_2d(b_dst, &tmB, &full[slot], kb * BK, 0);
-        } else {
-          for (int a = 0; a < b_atoms; ++a)
-            tma_load_2d(b_dst + a * 8192, &tmB, &full[slot], a * 64, kb * BK);
-        }
-        if (i == 0) QLORA_STAMP(2);
-        issued = i + 1;
-      }
-      if (*abort_flag) {
-        for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
-          mbar_drain(&full[j % STAGES], (j / STAGES) & 1);
-      }
-    }
-  } else if (warp == kMmaWarp) {
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(BM, BNp, A_MN, B_MN);
-      bool any = false;
-      for (int i = 0; i < nk; ++i) {
-        const int slot = i % STAGES;
-        const uint32_t ph = (i / STAGES) & 1;
-        if (!mbar_wait(&full[slot], ph, abort_flag)) break;
-        if (i == 0) QLORA_STAMP(3);
-        if (i == nk - 1) QLORA_STAMP(4);
-        tc_fence_after();
-        const uint32_t a_addr = smem_addr(smem + slot * SB);
-        const uint32_t b_addr = a_addr + A_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t ad = A_MN ? sw128_desc(a_addr + kk * 2048, 8192, 1024)
-                                   : sw128_desc(a_addr + kk * 32, 16, 1024);
-          const uint64_t bd = B_MN ? sw128_desc(b_addr + kk * 2048, 8192, 1024)
-                                   : sw128_desc(b_addr + kk * 32, 16, 1024);
-          umma_bf16(tmem_base, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&empty[slot]);
-        any = true;
-      }
-      umma_commit(acc_full);
-      if (*abort_flag && any) mbar_drain(acc_full, 0);
-    }
-  } else {
-    // ---------------- epilogue warps 0-3: one accumulator row per thread ------------------
-    const bool ok = (nk > 0) && mbar_wait(acc_full, 0, abort_flag);
-    if (threadIdx.x == 0) QLORA_STAMP(5);
-    tc_fence_after();
-    if (ok && !*abort_flag) {
-      const int row = m0 + warp * 32 + lane;
-      const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
-      const bool direct_bf16 = args.out_mode == kOutRoundBf16 && args.splits == 1;
-      // one accumulator chunk of 16 columns -> the output mode's destination
-      auto emit = [&](const uint32_t (&v)[16], int n0) {
-        if (row >= args.M || n0 >= args.Ncols) return;  // Ncols is a multiple of 16
-        if (args.out_mode == kOutAtomicTransposed) {
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            atomicAdd(args.out32 + static_cast<int64_t>(n0 + e) * args.ld + row,
-                      __uint_as_float(v[e]));
-        } else if (direct_bf16) {
-          const float a = args.alpha;
-          uint4 o0, o1;
-          o0.x = pack_bf16x2(a * __uint_as_float(v[0]), a * __uint_as_float(v[1]));
-          o0.y = pack_bf16x2(a * __uint_as_float(v[2]), a * __uint_as_float(v[3]));
-          o0.z = pack_bf16x2(a * __uint_as_float(v[4]), a * __uint_as_float(v[5]));
-          o0.w = pack_bf16x2(a * __uint_as_float(v[6]), a * __uint_as_float(v[7]));
-          o1.x = pack_bf16x2(a * __uint_as_float(v[8]), a * __uint_as_float(v[9]));
-          o1.y = pack_bf16x2(a * __uint_as_float(v[10]), a * __uint_as_float(v[11]));
-          o1.z = pack_bf16x2(a * __uint_as_float(v[12]), a * __uint_as_float(v[13]));
-          o1.w = pack_bf16x2(a * __uint_as_float(v[14]), a * __uint_as_float(v[15]));
-          const int64_t off = static_cast<int64_t>(row) * args.Ncols + n0;
-          reinterpret_cast<uint4*>(args.out16a + off)[0] = o0;
-          reinterpret_cast<uint4*>(args.out16a + off)[1] = o1;
-          if (args.out16b) {
-            reinterpret_cast<uint4*>(args.out16b + off)[0] = o0;
-            reinterpret_cast<uint4*>(args.out16b + off)[1] = o1;
-          }
-        } else {
-          float* dst = args.out32 + static_cast<int64_t>(row) * args.ld + n0;
-#pragma unroll
-          for (int e = 0; e < 16; e += 4)
-            red_add_v4(dst + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                       __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
-        }
-      };
-      // up to four 16-column TMEM loads in flight before one wait (the counts are warp-uniform)
-      const int nchunks = BNp / 16;
-      for (int c = 0; c < nchunks; c += 4) {
-        uint32_t v0[16], v1[16], v2[16], v3[16];
-        tmem_ld_16(lane_addr + c * 16, v0);
-        if (c + 1 < nchunks) tmem_ld_16(lane_addr + (c + 1) * 16, v1);
-        if (c + 2 < nchunks) tmem_ld_16(lane_addr + (c + 2) * 16, v2);
-        if (c + 3 < nchunks) tmem_ld_16(lane_addr + (c + 3) * 16, v3);
-        tmem_ld_wait();
-        emit(v0, c * 16);
-        if (c + 1 < nchunks) emit(v1, (c + 1) * 16);
-        if (c + 2 < nchunks) emit(v2, (c + 2) * 16);
-        if (c + 3 < nchunks) emit(v3, (c + 3) * 16);
-      }
-      // partial sums must be visible device-wide before this CTA is counted as arrived
-      if (args.out_mode == kOutRoundBf16 && args.splits > 1) __threadfence();
-    }
-    if (threadIdx.x == 0) QLORA_STAMP(6);
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == kMmaWarp) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, tmem_cols);
-  }
-  // kOutRoundBf16 with split-K: the last CTA of this M tile to finish converts the summed
-  // fp32 rows to bf16(alpha * sum). Nobody waits on anybody: earlier CTAs just exit.
-  if (args.out_mode == kOutRoundBf16 && args.splits > 1 && nk > 0) {
-    if (threadIdx.x == 0) {
-      __threadfence();
-      const unsigned prev = atomicAdd(args.counters + blockIdx.y, 1u);
-      last_flag = (prev == static_cast<unsigned>(args.splits - 1)) ? 1u : 0u;
-      __threadfence();
-    }
-    __syncthreads();
-    if (last_flag && warp < 4 && !*abort_flag) {
-      const int row = m0 + warp * 32 + lane;
-      if (row < args.M) {
-        const float* src = args.out32 + static_cast<int64_t>(row) * args.Ncols;
-        uint16_t* da = args.out16a + static_cast<int64_t>(row) * args.Ncols;
-        uint16_t* db = args.out16b ? args.out16b + static_cast<int64_t>(row) * args.Ncols : nullptr;
-        // 64 columns (16 independent 16-byte loads) in flight per round
-        for (int n0 = 0; n0 < args.Ncols; n0 += 64) {
-          float4 x[16];
-#pragma unroll
-          for (int u = 0; u < 16; ++u)
-            if (n0 + 4 * u < args.Ncols)
-              x[u] = __ldcg(reinterpret_cast<const float4*>(src + n0 + 4 * u));
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            if (n0 + 4 * u >= args.Ncols) break;
-            uint2 o;
-            o.x = pack_bf16x2(args.alpha * x[u].x, args.alpha * x[u].y);
-            o.y = pack_bf16x2(args.alpha * x[u].z, args.alpha * x[u].w);
-            *reinterpret_cast<uint2*>(da + n0 + 4 * u) = o;
-            if (db) *reinterpret_cast<uint2*>(db + n0 + 4 * u) = o;
-          }
-        }
-      }
-    }
-  }
-  if (threadIdx.x == 0) QLORA_STAMP(7);
 }
 
 }  // namespace qlora

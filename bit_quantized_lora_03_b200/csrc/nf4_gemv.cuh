@@ -510,14 +510,6 @@ constexpr size_t smem_bytes(int t, int r) {
 }
 }  // namespace gd
 
-__device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t rank) {
-  uint32_t raddr;
-  float v;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(raddr) : "r"(smem_addr(local)), "r"(rank));
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(raddr) : "memory");
-  return v;
-}
-
 __global__ void __cluster_dims__(gd::kClusterCtas, 1, 1) __launch_bounds__(gd::kThreads)
     gemv_lora_down_kernel(const uint16_t* __restrict__ X, const uint16_t* __restrict__ L1,
                           float* Tpart, float* Y32, unsigned* tile_cnt, int64_t h, int64_t o,

@@ -17,6 +17,7 @@
 
 #include "nf4_codec.cuh"
 #include "nf4_gemm.cuh"
+#include "tc_gemm.cuh"
 #include "nf4_gemv.cuh"
 
 using namespace qlora;
@@ -310,6 +311,8 @@ constexpr int64_t kGemvMaxTokens = 16;
 // ------------------------------------------------------------------------------------------
 // launch helpers
 // ------------------------------------------------------------------------------------------
+constexpr int kMaxTcSplits = 8;
+
 struct TcPlan {
   int stages, splits, kb_per_split, num_kb, mtiles, BNp;
   size_t smem;
@@ -331,6 +334,7 @@ TcPlan plan_tc(int64_t M, int64_t ncols, int64_t K, bool b_mn, int sms) {
   p.smem = tcg::smem_bytes(stages, p.BNp, b_mn);
   int splits = std::max(1, sms / p.mtiles);
   splits = std::min(splits, std::max(1, p.num_kb / 4));
+  splits = std::min(splits, kMaxTcSplits);  // split-K is one cluster (portable size)
 #ifdef QLORA_TUNING
   if (const char* e = std::getenv("QLORA_TC_WAVE")) splits = std::max(1, (std::atoi(e) * sms) / p.mtiles);
   if (const char* e = std::getenv("QLORA_TC_MINKB")) splits = std::min(splits, std::max(1, p.num_kb / std::atoi(e)));
@@ -339,6 +343,10 @@ TcPlan plan_tc(int64_t M, int64_t ncols, int64_t K, bool b_mn, int sms) {
     p.smem = tcg::smem_bytes(p.stages, p.BNp, b_mn);
   }
 #endif
+  // the split-K partial tile (128 rows of BNp + 4 floats) reuses the drained stage buffers
+  if (static_cast<size_t>(tcg::BM) * (p.BNp + 4) * 4 >
+      static_cast<size_t>(p.stages) * tcg::stage_bytes(p.BNp, b_mn))
+    splits = 1;
   p.kb_per_split = (p.num_kb + splits - 1) / splits;
   p.splits = (p.num_kb + p.kb_per_split - 1) / p.kb_per_split;
   return p;
@@ -347,7 +355,7 @@ TcPlan plan_tc(int64_t M, int64_t ncols, int64_t K, bool b_mn, int sms) {
 template <bool A_MN, bool B_MN>
 int launch_tc_gemm(const CUtensorMap& mA, const CUtensorMap& mB, int64_t M, int64_t ncols,
                    const TcPlan& pl, float alpha, int mode, float* out32, int64_t ld,
-                   uint16_t* o16a, uint16_t* o16b, unsigned* counters, cudaStream_t st) {
+                   uint16_t* o16a, uint16_t* o16b, cudaStream_t st) {
   TcGemmArgs a{};
   a.M = static_cast<int>(M);
   a.Ncols = static_cast<int>(ncols);
@@ -362,11 +370,26 @@ int launch_tc_gemm(const CUtensorMap& mA, const CUtensorMap& mB, int64_t M, int6
   a.ld = ld;
   a.out16a = o16a;
   a.out16b = o16b;
-  a.counters = counters;
-  dim3 grid(1, pl.mtiles, pl.splits);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1, static_cast<unsigned>(pl.mtiles), static_cast<unsigned>(pl.splits));
+  cfg.blockDim = dim3(tcg::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;  // the split-K CTAs of a tile: one cluster
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = static_cast<unsigned>(pl.splits);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
   {
     prof::Scope ps(prof::kTcGemm, st);
-    tc_gemm_kernel<A_MN, B_MN><<<grid, tcg::kThreads, pl.smem, st>>>(mA, mB, a);
+    e = cudaLaunchKernelEx(&cfg, tc_gemm_kernel<A_MN, B_MN>, mA, mB, a);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
   }
   return launch_status();
 }
@@ -418,25 +441,21 @@ int launch_nf4_gemm(const CUtensorMap& mA, const CUtensorMap& mP, const CUtensor
 }
 
 // out16 = bf16(s . A.B) (and out16b if given) for a rank-r down projection: A is t x K
-// (K-major), B given by its map (ncols = r). One launch; with split-K the partial sums meet
-// in ws.acc32 and the last CTA of each 128-token tile rounds them.
+// (K-major), B given by its map (ncols = r). One launch; split-K CTAs of a tile form one
+// cluster and reduce through distributed shared memory.
 template <bool B_MN>
 int lora_down(const CUtensorMap& mA, const CUtensorMap& mB, int64_t t, int64_t K, int64_t r,
-              float s, const LoraWs& ws, uint16_t* out16, uint16_t* out16b, int sms,
-              cudaStream_t st) {
+              float s, uint16_t* out16, uint16_t* out16b, int sms, cudaStream_t st) {
   TcPlan pl = plan_tc(t, r, K, B_MN, sms);
 #ifdef QLORA_TUNING
   if (const char* e = std::getenv("QLORA_RB_SPLITS")) {
-    int sp = std::max(1, std::min(pl.num_kb, std::atoi(e)));
+    int sp = std::max(1, std::min({pl.num_kb, kMaxTcSplits, std::atoi(e)}));
     pl.kb_per_split = (pl.num_kb + sp - 1) / sp;
     pl.splits = (pl.num_kb + pl.kb_per_split - 1) / pl.kb_per_split;
   }
 #endif
-  if (pl.splits > 1 &&
-      cudaMemsetAsync(ws.acc32, 0, lora_acc_bytes(t, r) + lora_counter_bytes(t), st) != cudaSuccess)
-    return QLORA_ERR_CUDA;
-  return launch_tc_gemm<false, B_MN>(mA, mB, t, r, pl, s, kOutRoundBf16, ws.acc32, r, out16,
-                                     out16b, ws.counters, st);
+  return launch_tc_gemm<false, B_MN>(mA, mB, t, r, pl, s, kOutRoundBf16, nullptr, r, out16,
+                                     out16b, st);
 }
 
 }  // namespace
@@ -676,7 +695,7 @@ int qlora_linear_fwd(const uint16_t* X, int64_t t, const nf4_weight* W, const ui
 
 
   uint16_t* sT = ws.b16;
-  if ((rc = lora_down<true>(mX, mL1, t, h, r, s, ws, sT, sT_out, sms, st))) return rc;
+  if ((rc = lora_down<true>(mX, mL1, t, h, r, s, sT, sT_out, sms, st))) return rc;
 
   // Y = X . W' + sT . L2
   CUtensorMap mA, mP, mA2, mB2;
@@ -725,14 +744,14 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t t, const nf4
       !map_bf16(&mL2k, L2, o, r, 64, static_cast<uint32_t>((r + 15) / 16 * 16)))
     return QLORA_ERR_CUDA;
   uint16_t* sU = wsU.b16;
-  if ((rc = lora_down<false>(mdY, mL2k, t, o, r, s, wsU, sU, nullptr, sms, st))) return rc;
+  if ((rc = lora_down<false>(mdY, mL2k, t, o, r, s, sU, nullptr, sms, st))) return rc;
 
   // sT = bf16(s . X . L1) unless the forward's copy was passed in
   const uint16_t* sT = sT_saved;
   if (!sT) {
     CUtensorMap mX, mL1;
     if (!map_bf16(&mX, X, h, t, 64, 128) || !map_bf16(&mL1, L1, r, h, 64, 64)) return QLORA_ERR_CUDA;
-    if ((rc = lora_down<true>(mX, mL1, t, h, r, s, wsT, wsT.b16, nullptr, sms, st))) return rc;
+    if ((rc = lora_down<true>(mX, mL1, t, h, r, s, wsT.b16, nullptr, sms, st))) return rc;
     sT = wsT.b16;
   }
 
@@ -757,20 +776,17 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t t, const nf4
   }
 
   // dL1 = X^T . sU (h x r) and dL2^T = dY^T . sT (o x r), reductions over the t tokens
-  if (cudaMemsetAsync(dL1, 0, static_cast<size_t>(h) * r * 4, st) != cudaSuccess ||
-      cudaMemsetAsync(dL2, 0, static_cast<size_t>(r) * o * 4, st) != cudaSuccess)
-    return QLORA_ERR_CUDA;
   CUtensorMap mXmn, msU, mdYmn, msT;
   if (!map_bf16(&mXmn, X, h, t, 64, 64) || !map_bf16(&msU, sU, r, t, 64, 64) ||
       !map_bf16(&mdYmn, dY, o, t, 64, 64) || !map_bf16(&msT, sT, r, t, 64, 64))
     return QLORA_ERR_CUDA;
   const TcPlan p1 = plan_tc(h, r, t, true, sms);
-  if ((rc = launch_tc_gemm<true, true>(mXmn, msU, h, r, p1, 1.0f, kOutAtomicRowMajor, dL1, r,
-                                       nullptr, nullptr, nullptr, st)))
+  if ((rc = launch_tc_gemm<true, true>(mXmn, msU, h, r, p1, 1.0f, kOutRowMajor, dL1, r,
+                                       nullptr, nullptr, st)))
     return rc;
   const TcPlan p2 = plan_tc(o, r, t, true, sms);
-  return launch_tc_gemm<true, true>(mdYmn, msT, o, r, p2, 1.0f, kOutAtomicTransposed, dL2, o,
-                                    nullptr, nullptr, nullptr, st);
+  return launch_tc_gemm<true, true>(mdYmn, msT, o, r, p2, 1.0f, kOutTransposed, dL2, o,
+                                    nullptr, nullptr, st);
 }
 
 }  // extern "C"
