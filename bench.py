@@ -200,6 +200,22 @@ def timed(fn, steps, warmup, world, dev):
     return dp.max_over_ranks(start.elapsed_time(end), dev)
 
 
+def queued_ms(fn, reps, warmup):
+    """Device time of `reps` calls of fn queued behind a device-side sleep, so that the events
+    time back-to-back GPU work rather than the host's launch rate (single GPU legs)."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    torch.cuda._sleep(QUEUE_SLEEP_CYCLES)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(reps):
+        fn()
+    end.record()
+    torch.cuda.synchronize()
+    return start.elapsed_time(end)
+
+
 def fused_gemm_flops(layers):
     """Algorithmic flops of the fused NF4 GEMM launches of one step: forward X.W' + sT.L2 and
     backward dY.W'^T + sU.L1^T, per linear."""
@@ -296,8 +312,8 @@ def codec_leg(dev, peaks):
     def deq():
         for p, o_ in zip(packs, outs):
             B.nf4_dequantize(p, out=o_)
-    qms = timed(quant, 5, 2, 1, dev) / 5
-    dms = timed(deq, 5, 2, 1, dev) / 5
+    qms = queued_ms(quant, 5, 2) / 5
+    dms = queued_ms(deq, 5, 2) / 5
     qbytes = 4 * n + packed
     dbytes = packed + 2 * n
     res = {

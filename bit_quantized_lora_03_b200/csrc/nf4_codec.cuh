@@ -34,54 +34,146 @@ __device__ __forceinline__ uint32_t nf4_code_of(float w, float c1, const float* 
   return c;
 }
 
-// One CTA of 256 threads per group of 256 blocks (16384 weights), grid-stride over groups.
-// Half-warp h16 of iteration `it` owns block it*16 + h16; each thread loads one float4.
-__global__ void __launch_bounds__(256) nf4_quantize_kernel(const float* __restrict__ W,
-                                                           uint8_t* __restrict__ codes,
-                                                           uint8_t* __restrict__ q8,
-                                                           float* __restrict__ s2,
-                                                           int64_t nblocks, Nf4Table tab) {
+// The same decision without a division in the common case. x' = w * RN(1/c1) is within 2^-22
+// of the IEEE quotient x = RN(w / c1) for |w| <= c1 (two roundings of relative size 2^-24
+// each, |x| <= 1), so x' and x fall on the same side of every threshold farther than 2^-20
+// from x'. The thresholds are found through 128 equal buckets over [-1, 1): bucket b =
+// floor((x' + 1) * 64), read from the mantissa of x' + 3 (which lies in [2, 4)); each bucket
+// holds the count of thresholds below it and the one threshold inside it (or 4 if none).
+// When x' is within 2^-20 of that threshold, the code is decided on the IEEE quotient. The
+// host builds the buckets only if every bucket holds at most one threshold and no threshold
+// lies within 2^-18 of a bucket edge (so a bucket misread by rounding near an edge still
+// gives the same count); otherwise `exact_only` sends every weight to nf4_code_of.
+struct Nf4Buckets {
+  float thr[128];
+  float lo[128];  // counts, as floats
+  int exact_only;
+};
+
+__device__ __noinline__ uint32_t nf4_code_exact(float w, float c1, const float* mids) {
+  return nf4_code_of(w, c1, mids);
+}
+
+// Fast decision; sets `near` when x' is within 2^-20 of the bucket's threshold (the caller
+// then decides on the IEEE quotient). The bucket table holds one copy per lane (entry b of
+// lane l at 256 b + 8 l: {threshold, count as integer bits}), so lookups never collide on a bank.
+__device__ __forceinline__ uint32_t nf4_code_fast(float w, float r, uint32_t lane_tab, bool& near) {
+  const float x = __fmul_rn(w, r);
+  const float xc = fminf(fmaxf(x, -1.0f), 1.0f - 0x1p-22f);  // then xc + 3 <= 4 - 2^-22 exactly
+  const uint32_t b = (__float_as_uint(__fadd_rn(xc, 3.0f)) >> 16) & 127u;
+  float thr;
+  uint32_t lo;
+  asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(thr), "=r"(lo) : "r"(lane_tab + b * 256u));
+  near |= fabsf(__fsub_rn(x, thr)) < 0x1p-20f;
+  return lo + (x > thr ? 1u : 0u);
+}
+
+// max that propagates NaN (so a block's absmax is NaN or inf exactly when it holds one)
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
+// Persistent: one CTA of 512 threads per SM walks the groups of 256 blocks (16384 weights,
+// 64 KB of fp32) g = blockIdx.x, blockIdx.x + gridDim.x, ...; thread 0 streams each group
+// into one of two 64 KB shared-memory buffers with bulk copies, one group ahead, so HBM reads
+// overlap the previous group's arithmetic. Half-warp h of pass p (0..7) owns block 32p + h;
+// each of its lanes reads one float4 of the block from shared memory.
+namespace qz {
+constexpr int kThreads = 512;
+constexpr int kGroupBytes = kGroup * kBlock * 4;  // 64 KB
+constexpr int kChunk = 16384;                       // bytes per bulk copy
+constexpr size_t smem_bytes() { return 2 * static_cast<size_t>(kGroupBytes) + 64; }
+}  // namespace qz
+
+__global__ void __launch_bounds__(qz::kThreads, 1) nf4_quantize_kernel(
+    const float* __restrict__ W, uint8_t* __restrict__ codes, uint8_t* __restrict__ q8,
+    float* __restrict__ s2, int64_t nblocks, Nf4Table tab, Nf4Buckets bkt) {
+  extern __shared__ __align__(128) uint8_t qsm[];
   __shared__ float mids[16];
+  __shared__ __align__(16) float2 bk[128 * 32];  // [bucket][lane]
   __shared__ float c1s[kGroup];
-  __shared__ float wmax[8];
+  __shared__ float wmax[qz::kThreads / 32];
+  __shared__ uint32_t abort_flag;
+  float* buf = reinterpret_cast<float*>(qsm);                        // [2][16384]
+  uint64_t* full = reinterpret_cast<uint64_t*>(qsm + 2 * qz::kGroupBytes);
   const int tid = threadIdx.x;
   if (tid < 16) mids[tid] = tab.mid[tid];
-  __syncthreads();
-  const int h16 = tid >> 4, l16 = tid & 15;
+  for (int i = tid; i < 128 * 32; i += qz::kThreads)
+    bk[i] = make_float2(bkt.thr[i >> 5], __uint_as_float(static_cast<uint32_t>(bkt.lo[i >> 5])));
+  const bool fast = bkt.exact_only == 0;
+  const uint32_t lane_tab = smem_addr(bk) + static_cast<uint32_t>(tid & 31) * 8u;
+  const int h32 = tid >> 4, l16 = tid & 15;
   const int64_t ngroups = (nblocks + kGroup - 1) / kGroup;
   bool bad = false;
 
-  for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x) {
-    const int nb = static_cast<int>((nblocks - g * kGroup < kGroup ? nblocks - g * kGroup : kGroup));
-    const float* base = W + g * (kGroup * kBlock);
-    float4 v[16];
+  auto group_bytes = [&](int64_t g) {
+    const int64_t nb = nblocks - g * kGroup < kGroup ? nblocks - g * kGroup : kGroup;
+    return static_cast<uint32_t>(nb * kBlock * 4);
+  };
+  auto issue = [&](int64_t g, int b) {  // thread 0: stream group g into buffer b
+    const uint32_t bytes = group_bytes(g);
+    mbar_arrive_expect_tx(&full[b], bytes);
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(W + g * (kGroup * kBlock));
+    uint8_t* dst = reinterpret_cast<uint8_t*>(buf + b * (kGroup * kBlock));
+    for (uint32_t off = 0; off < bytes; off += qz::kChunk)
+      bulk_load(dst + off, src + off, bytes - off < qz::kChunk ? bytes - off : qz::kChunk, &full[b]);
+  };
+  if (tid == 0) {
+    abort_flag = 0u;
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
+    fence_mbar_init();
+    if (blockIdx.x < ngroups) issue(blockIdx.x, 0);
+    if (blockIdx.x + gridDim.x < ngroups) issue(blockIdx.x + gridDim.x, 1);
+  }
+  __syncthreads();
+
+  int it = 0;
+  for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x, ++it) {
+    const int b = it & 1;
+    const int nb = static_cast<int>(group_bytes(g) / (kBlock * 4));
+    if (!mbar_wait(&full[b], static_cast<uint32_t>(it >> 1) & 1u, &abort_flag)) break;
+    const float* gb = buf + b * (kGroup * kBlock);
 #pragma unroll
-    for (int it = 0; it < 16; ++it) {
-      if (it * 16 + h16 < nb)
-        v[it] = __ldcs(reinterpret_cast<const float4*>(base + it * 1024 + tid * 4));
-      else
-        v[it] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll
-    for (int it = 0; it < 16; ++it) {
-      const int blk = it * 16 + h16;
-      const float4 x = v[it];
-      bad |= !(isfinite(x.x) && isfinite(x.y) && isfinite(x.z) && isfinite(x.w));
-      float a = fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w)));
-      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 8));
-      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
-      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
-      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+    for (int p = 0; p < kGroup / 32; ++p) {
+      const int blk = p * 32 + h32;
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (blk < nb) x = *reinterpret_cast<const float4*>(gb + blk * kBlock + l16 * 4);
+      float a = fmax_nan(fmax_nan(fabsf(x.x), fabsf(x.y)), fmax_nan(fabsf(x.z), fabsf(x.w)));
+      a = fmax_nan(a, __shfl_xor_sync(0xffffffffu, a, 8));
+      a = fmax_nan(a, __shfl_xor_sync(0xffffffffu, a, 4));
+      a = fmax_nan(a, __shfl_xor_sync(0xffffffffu, a, 2));
+      a = fmax_nan(a, __shfl_xor_sync(0xffffffffu, a, 1));
+      bad |= !(a <= 3.402823466e38f);  // the block holds a NaN or an infinity
       if (blk < nb) {
         if (l16 == 0) c1s[blk] = a;
-        const uint32_t k0 = nf4_code_of(x.x, a, mids), k1 = nf4_code_of(x.y, a, mids);
-        const uint32_t k2 = nf4_code_of(x.z, a, mids), k3 = nf4_code_of(x.w, a, mids);
+        uint32_t k0, k1, k2, k3;
+        bool near = !(fast && a >= 0x1p-120f);  // RN(1/c1) finite and normal
+        if (!near) {
+          const float rc = __frcp_rn(a);
+          k0 = nf4_code_fast(x.x, rc, lane_tab, near);
+          k1 = nf4_code_fast(x.y, rc, lane_tab, near);
+          k2 = nf4_code_fast(x.z, rc, lane_tab, near);
+          k3 = nf4_code_fast(x.w, rc, lane_tab, near);
+        }
+        if (near) {  // rare: some weight lies next to a threshold, or c1 is tiny
+          k0 = nf4_code_exact(x.x, a, mids);
+          k1 = nf4_code_exact(x.y, a, mids);
+          k2 = nf4_code_exact(x.z, a, mids);
+          k3 = nf4_code_exact(x.w, a, mids);
+        }
         const uint32_t packed = ((k0 << 4) | k1) | (((k2 << 4) | k3) << 8);
-        *reinterpret_cast<uint16_t*>(codes + g * (kGroup * kBlock / 2) + it * 512 + tid * 2) =
+        *reinterpret_cast<uint16_t*>(codes + g * (kGroup * kBlock / 2) + blk * 32 + l16 * 2) =
             static_cast<uint16_t>(packed);
       }
     }
-    __syncthreads();
+    __syncthreads();  // every thread is done with buffer b and has written its c1s
+    if (tid == 0 && g + 2 * static_cast<int64_t>(gridDim.x) < ngroups) {
+      fence_proxy_async_smem();  // the reads above come before the copy that overwrites b
+      issue(g + 2 * static_cast<int64_t>(gridDim.x), b);
+    }
     // second level: c2 = max over the group's block scales; s2 = c2 / 255; q8 = rint(c1 / s2)
     const float c1 = (tid < nb) ? c1s[tid] : 0.0f;
     float m = c1;
@@ -91,7 +183,7 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const float* __restri
     __syncthreads();
     float c2 = wmax[0];
 #pragma unroll
-    for (int i = 1; i < 8; ++i) c2 = fmaxf(c2, wmax[i]);
+    for (int i = 1; i < qz::kThreads / 32; ++i) c2 = fmaxf(c2, wmax[i]);
     const float sc = __fdiv_rn(c2, 255.0f);
     if (tid < nb) {
       int qv = 0;
@@ -99,7 +191,7 @@ __global__ void __launch_bounds__(256) nf4_quantize_kernel(const float* __restri
       q8[g * kGroup + tid] = static_cast<uint8_t>(qv);
     }
     if (tid == 0) s2[g] = sc;
-    __syncthreads();
+    __syncthreads();  // c1s and wmax are rewritten by the next group
   }
   if (bad) report(kDevNonfinite);
 }

@@ -85,6 +85,28 @@ Nf4Table device_table() {
   return t;
 }
 
+// Buckets of the quantizer's fast decision (see nf4_code_fast): bucket b covers
+// [-1 + b/64, -1 + (b+1)/64); fp32 arithmetic on these edges is exact.
+Nf4Buckets device_buckets() {
+  Nf4Buckets bk{};
+  const Codebook& cb = codebook();
+  int bad = 0;
+  for (int b = 0; b < 128; ++b) {
+    const float lo = -1.0f + static_cast<float>(b) / 64.0f, hi = lo + 1.0f / 64.0f;
+    int n = 0;
+    while (n < 15 && cb.mid[n] < lo) ++n;
+    bk.lo[b] = static_cast<float>(n);
+    bk.thr[b] = (n < 15 && cb.mid[n] < hi) ? cb.mid[n] : 4.0f;
+    if (n + 1 < 15 && cb.mid[n + 1] < hi) bad = 1;  // two thresholds in one bucket
+  }
+  for (int i = 0; i < 15; ++i) {  // no threshold within 2^-18 of a bucket edge
+    const double u = (static_cast<double>(cb.mid[i]) + 1.0) * 64.0;
+    if (std::fabs(u - std::nearbyint(u)) / 64.0 < std::ldexp(1.0, -18)) bad = 1;
+  }
+  bk.exact_only = bad;
+  return bk;
+}
+
 // ------------------------------------------------------------------------------------------
 // device checks, kernel attributes
 // ------------------------------------------------------------------------------------------
@@ -124,6 +146,8 @@ int current_device(int* dev_out) {
                                  static_cast<int>(tc::nf4_gemm_smem_bytes())) == cudaSuccess;
     fine &= cudaFuncSetAttribute(nf4_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(tc::nf4_gemm_smem_bytes())) == cudaSuccess;
+    fine &= cudaFuncSetAttribute(nf4_quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(qz::smem_bytes())) == cudaSuccess;
     fine &= cudaFuncSetAttribute(gemv_lora_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(gd::smem_bytes(16, 256))) == cudaSuccess;
     fine &= cudaFuncSetAttribute(nf4_gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -584,11 +608,11 @@ int nf4_quantize(const float* Wt, const nf4_weight* q, qlora_stream_t stream) {
   if ((rc = current_device(&dev))) return rc;
   const int64_t nblocks = q->out_features * q->in_features / 64;
   const int64_t ngroups = (nblocks + 255) / 256;
-  const int grid = static_cast<int>(std::min<int64_t>(ngroups, int64_t(sm_count(dev)) * 4));
+  const int grid = static_cast<int>(std::min<int64_t>(ngroups, int64_t(sm_count(dev))));
   {
     prof::Scope ps(prof::kQuant, reinterpret_cast<cudaStream_t>(stream));
-    nf4_quantize_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        Wt, q->codes, q->absmax_q8, q->absmax_s2, nblocks, device_table());
+    nf4_quantize_kernel<<<grid, qz::kThreads, qz::smem_bytes(), reinterpret_cast<cudaStream_t>(stream)>>>(
+        Wt, q->codes, q->absmax_q8, q->absmax_s2, nblocks, device_table(), device_buckets());
   }
   return launch_status();
 }

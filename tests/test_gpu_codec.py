@@ -52,6 +52,31 @@ def test_llama7b_layer_with_outliers(i):
     _check_full(inputs.weight_f32(o, h, 200 + i, outliers=True))
 
 
+def test_weights_next_to_thresholds():
+    """Blocks whose weights sit within a few ulps of c1 x (each threshold), plus +-c1 itself,
+    over block scales from subnormal to 1e3: the quantizer's reciprocal fast path must hand
+    every such weight to the IEEE quotient and agree with the oracle bit for bit."""
+    mids = O.nf4_midpoints().astype(np.float32)
+    rng = np.random.default_rng(7)
+    rows = []
+    for c1 in np.concatenate([np.float32([1.0, 1e-39, 3e-41, 2.5e-38]),
+                              np.exp(rng.uniform(-60, 7, 60)).astype(np.float32)]):
+        c1 = np.float32(c1)
+        vals = [c1, -c1]
+        for m in mids:
+            v = np.float32(m * c1)
+            for k in range(-3, 4):
+                u = v
+                for _ in range(abs(k)):
+                    u = np.nextafter(u, np.float32(np.inf) if k > 0 else np.float32(-np.inf))
+                vals.append(np.clip(u, -c1, c1))
+        vals = np.array(vals, np.float32)
+        row = np.resize(vals, 64 * ((vals.size + 63) // 64)).astype(np.float32)
+        row[::64] = c1   # every block's absmax is exactly c1
+        rows.append(np.resize(row, 64 * 4))
+    _check_full(torch.from_numpy(np.stack(rows).astype(np.float32)))
+
+
 def test_decode_weight_4096x11008():
     _check_full(inputs.decode_gemv_weights()[0][1])
 
