@@ -13,9 +13,10 @@
 //    the forward (rows of Wt are N), MN-major for the backward (rows of Wt are K). A pair of
 //    CTAs (a cluster of 2) owns 512 tokens x 256 columns and issues tcgen05.mma.cta_group::2:
 //    each CTA dequantizes only its 128 of the 256 columns, and two accumulators per CTA (all
-//    512 TMEM columns) make every dequantized tile feed 512 tokens. The r/64 LoRA K-steps
-//    (A = sT or sU, B = L2 or L1, both by TMA) run first, then the h/64 (or o/64) weight
-//    K-steps. The same 8 warps then drain TMEM to bf16.
+//    512 TMEM columns) make every dequantized tile feed 512 tokens. The h/64 (or o/64) weight
+//    K-steps run first, then the r/64 LoRA K-steps (A = sT or sU, B = L2 or L1, both by
+//    TMA), so that the kernel can start, by programmatic dependent launch, while the kernel
+//    that produces sT or sU is still running. The same 8 warps then drain TMEM to bf16.
 //
 // (tc_gemm.cuh holds the plain tcgen05 GEMM for the rank-r products.)
 //
@@ -134,7 +135,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   const int n0 = blockIdx.y * BN;                        // the pair's 256 output columns
   const int nh0 = n0 + static_cast<int>(rank) * BNH;    // this CTA's 128 of them
   const int mrow = (blockIdx.x >> 1) * PAIR_M + static_cast<int>(rank) * 128;  // + a * 256
-  const int total = args.num_lkb + args.num_kb;
+  const int total = args.num_kb + args.num_lkb;   // weight K-steps, then the LoRA K-steps
+  pdl_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -173,20 +175,24 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         if (!mbar_wait(&empty[slot], ph ^ 1u, abort_flag)) break;
         uint8_t* a_dst = sA + slot * A_BYTES;
         uint8_t* b_dst = sB + slot * B_BYTES;
-        if (i < args.num_lkb) {
+        if (i >= args.num_kb) {
+          // sT / sU come from the kernel launched just before this one, which may still be
+          // running (programmatic dependent launch): wait for it before the first LoRA load
+          if (i == args.num_kb) pdl_wait();
+          const int li = i - args.num_kb;
           mbar_arrive_expect_tx(&full_ap[slot], A_BYTES + B_BYTES);
-          tma_load_2d(a_dst, &tmA2, &full_ap[slot], i * BK, mrow);
-          tma_load_2d(a_dst + A_HALF, &tmA2, &full_ap[slot], i * BK, mrow + 256);
+          tma_load_2d(a_dst, &tmA2, &full_ap[slot], li * BK, mrow);
+          tma_load_2d(a_dst + A_HALF, &tmA2, &full_ap[slot], li * BK, mrow + 256);
           if (!kBwd) {
             // L2 (r x o), MN-major B: this CTA's two 64-column atoms, 8 KB apart
-            tma_load_2d(b_dst, &tmB2, &full_ap[slot], nh0, i * BK);
-            tma_load_2d(b_dst + 8192, &tmB2, &full_ap[slot], nh0 + 64, i * BK);
+            tma_load_2d(b_dst, &tmB2, &full_ap[slot], nh0, li * BK);
+            tma_load_2d(b_dst + 8192, &tmB2, &full_ap[slot], nh0 + 64, li * BK);
           } else {
             // L1 (h x r), K-major B: this CTA's 128 rows of 64 ranks
-            tma_load_2d(b_dst, &tmB2, &full_ap[slot], i * BK, nh0);
+            tma_load_2d(b_dst, &tmB2, &full_ap[slot], li * BK, nh0);
           }
         } else {
-          const int kb = i - args.num_lkb;
+          const int kb = i;
           mbar_arrive_expect_tx(&full_ap[slot], A_BYTES + P_BYTES);
           tma_load_2d(a_dst, &tmA, &full_ap[slot], kb * BK, mrow);
           tma_load_2d(a_dst + A_HALF, &tmA, &full_ap[slot], kb * BK, mrow + 256);
@@ -218,7 +224,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         if (!mbar_wait(&full_b[slot], ph, abort_flag)) break;
         if (!mbar_wait_cluster(&peer_ready[slot], ph, abort_flag)) break;
         tc_fence_after();
-        const bool lora = i < args.num_lkb;
+        const bool lora = i >= args.num_kb;
         const bool b_mn = lora ? !kBwd : kBwd;
         const uint32_t idesc = lora ? kIdescLora : kIdescMain;
         const uint32_t a_addr = smem_addr(sA + slot * A_BYTES);
@@ -295,8 +301,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       const int slot = i % STAGES;
       const uint32_t ph = (i / STAGES) & 1;
       if (!mbar_wait(&empty[slot], ph ^ 1u, abort_flag)) { ok = false; break; }
-      if (i >= args.num_lkb) {
-        const int kb = i - args.num_lkb;
+      if (i < args.num_kb) {
+        const int kb = i;
         const float k = __fmul_rn(static_cast<float>(q_cur), s_cur);
         q_cur = q_nxt;
         s_cur = s_nxt;
@@ -361,6 +367,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     tc_fence_after();
     tmem_dealloc2(tmem_base, kTmemCols);
   }
+  // completion stays in stream order even when an abort skipped the wait before the LoRA steps
+  if (threadIdx.x == 0) pdl_wait();
 }
 
 }  // namespace qlora

@@ -168,6 +168,15 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Programmatic dependent launch. launch_dependents lets the next kernel on the stream (if it
+// was launched with programmatic stream serialization) be scheduled while this one still
+// runs; wait blocks until the previous kernel has completed and its memory is visible (a
+// no-op for a kernel launched without that attribute).
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Untiled bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned) from global
 // to shared memory, completing that many bytes of transaction count on `bar`.
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes,

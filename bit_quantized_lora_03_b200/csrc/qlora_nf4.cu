@@ -379,7 +379,7 @@ TcPlan plan_tc(int64_t M, int64_t ncols, int64_t K, bool b_mn, int sms) {
 template <bool A_MN, bool B_MN>
 int launch_tc_gemm(const CUtensorMap& mA, const CUtensorMap& mB, int64_t M, int64_t ncols,
                    const TcPlan& pl, float alpha, int mode, float* out32, int64_t ld,
-                   uint16_t* o16a, uint16_t* o16b, cudaStream_t st) {
+                   uint16_t* o16a, uint16_t* o16b, int pdl, cudaStream_t st) {
   TcGemmArgs a{};
   a.M = static_cast<int>(M);
   a.Ncols = static_cast<int>(ncols);
@@ -394,18 +394,21 @@ int launch_tc_gemm(const CUtensorMap& mA, const CUtensorMap& mB, int64_t M, int6
   a.ld = ld;
   a.out16a = o16a;
   a.out16b = o16b;
+  a.pdl = pdl;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(1, static_cast<unsigned>(pl.mtiles), static_cast<unsigned>(pl.splits));
   cfg.blockDim = dim3(tcg::kThreads, 1, 1);
   cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;  // the split-K CTAs of a tile: one cluster
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = static_cast<unsigned>(pl.splits);
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl == kPdlNone ? 1 : 2;
   cudaError_t e;
   {
     prof::Scope ps(prof::kTcGemm, st);
@@ -445,13 +448,17 @@ int launch_nf4_gemm(const CUtensorMap& mA, const CUtensorMap& mP, const CUtensor
   cfg.blockDim = dim3(tc::kThreads, 1, 1);
   cfg.dynamicSmemBytes = tc::nf4_gemm_smem_bytes();
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  // always launched right after the kernel that produces its LoRA operand (sT or sU): it
+  // may start early and waits for that kernel before its LoRA K-steps
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   cudaError_t e;
   {
     prof::Scope ps(prof_kind, st);
@@ -479,7 +486,7 @@ int lora_down(const CUtensorMap& mA, const CUtensorMap& mB, int64_t t, int64_t K
   }
 #endif
   return launch_tc_gemm<false, B_MN>(mA, mB, t, r, pl, s, kOutRoundBf16, nullptr, r, out16,
-                                     out16b, st);
+                                     out16b, kPdlNone, st);
 }
 
 }  // namespace
@@ -779,6 +786,20 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t t, const nf4
     sT = wsT.b16;
   }
 
+  // Launch order U [, sT], dL1, dX, dL2, each after the first by programmatic dependent
+  // launch: dL1 waits for sU; the fused dX kernel streams dY and W' while dL1 runs and waits
+  // for it (hence for sU) before its LoRA K-step; dL2 needs nothing made in this call unless
+  // sT was recomputed, so it can fill the SMs the dX kernel's last wave leaves idle.
+  // dL1 = X^T . sU (h x r) and dL2^T = dY^T . sT (o x r), reductions over the t tokens
+  CUtensorMap mXmn, msU, mdYmn, msT;
+  if (!map_bf16(&mXmn, X, h, t, 64, 64) || !map_bf16(&msU, sU, r, t, 64, 64) ||
+      !map_bf16(&mdYmn, dY, o, t, 64, 64) || !map_bf16(&msT, sT, r, t, 64, 64))
+    return QLORA_ERR_CUDA;
+  const TcPlan p1 = plan_tc(h, r, t, true, sms);
+  if ((rc = launch_tc_gemm<true, true>(mXmn, msU, h, r, p1, 1.0f, kOutRowMajor, dL1, r,
+                                       nullptr, nullptr, kPdlWaitFirst, st)))
+    return rc;
+
   // dX = dY . W'^T + sU . L1^T
   {
     CUtensorMap mA, mP, mA2, mB2;
@@ -799,18 +820,9 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t t, const nf4
     if ((rc = launch_nf4_gemm<true>(mA, mP, mA2, mB2, ga, t, h, st, prof::kGemmBwd))) return rc;
   }
 
-  // dL1 = X^T . sU (h x r) and dL2^T = dY^T . sT (o x r), reductions over the t tokens
-  CUtensorMap mXmn, msU, mdYmn, msT;
-  if (!map_bf16(&mXmn, X, h, t, 64, 64) || !map_bf16(&msU, sU, r, t, 64, 64) ||
-      !map_bf16(&mdYmn, dY, o, t, 64, 64) || !map_bf16(&msT, sT, r, t, 64, 64))
-    return QLORA_ERR_CUDA;
-  const TcPlan p1 = plan_tc(h, r, t, true, sms);
-  if ((rc = launch_tc_gemm<true, true>(mXmn, msU, h, r, p1, 1.0f, kOutRowMajor, dL1, r,
-                                       nullptr, nullptr, st)))
-    return rc;
   const TcPlan p2 = plan_tc(o, r, t, true, sms);
-  return launch_tc_gemm<true, true>(mdYmn, msT, o, r, p2, 1.0f, kOutTransposed, dL2, o,
-                                    nullptr, nullptr, st);
+  return launch_tc_gemm<true, true>(mdYmn, msT, o, r, p2, 1.0f, kOutTransposed, dL2, o, nullptr,
+                                    nullptr, sT_saved ? kPdlWaitLast : kPdlWaitFirst, st);
 }
 
 }  // extern "C"

@@ -46,6 +46,14 @@ enum TcOutMode : int {
 // leaves its fp32 partial tile in its own shared memory, and after a cluster barrier rank q
 // sums its share of the tile's rows over all ranks through distributed shared memory and
 // writes them. No global atomics, no zeroed accumulators, no arrival counters.
+// How a launch relates to the kernel before it on the stream (programmatic dependent launch):
+enum TcPdl : int {
+  kPdlNone = 0,       // launched normally: starts after all earlier work
+  kPdlWaitFirst = 1,  // may start early; reads nothing before the previous kernel completes
+  kPdlWaitLast = 2,   // may start early and needs nothing from the previous kernel; it still
+                      // completes only after it, so completion stays in stream order
+};
+
 struct TcGemmArgs {
   int M;
   int Ncols;         // real number of output columns (<= BNp, a multiple of 16)
@@ -60,6 +68,7 @@ struct TcGemmArgs {
   int64_t ld;
   uint16_t* out16a;
   uint16_t* out16b;
+  int pdl;           // TcPdl
 };
 
 #ifdef QLORA_TRACE
@@ -99,6 +108,7 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
   const uint32_t tmem_cols = BNp <= 32 ? 32u : (BNp <= 64 ? 64u : (BNp <= 128 ? 128u : 256u));
   const int b_atoms = (BNp + 63) / 64;
   const uint32_t bbytes = static_cast<uint32_t>(b_bytes(BNp, B_MN));
+  pdl_launch_dependents();
 
   if (threadIdx.x == 0) {
     QLORA_STAMP(0);
@@ -126,6 +136,7 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
 
   if (warp == kTmaWarp) {
     if (lane == 0) {
+      if (args.pdl == kPdlWaitFirst) pdl_wait();  // every global access follows the loads
       int issued = 0;
       for (int i = 0; i < nk; ++i) {
         const int slot = i % STAGES;
@@ -306,6 +317,7 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
     }
     cluster_sync();  // the partial tiles stay in place until every rank has read them
   }
+  if (args.pdl == kPdlWaitLast && threadIdx.x == 0) pdl_wait();
   if (threadIdx.x == 0) QLORA_STAMP(7);
 }
 
