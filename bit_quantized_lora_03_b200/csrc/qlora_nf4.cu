@@ -302,11 +302,8 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 // workspace region of one rank-r down projection (each part 256-byte aligned): the fp32
 // t x r split-K accumulator, one arrival counter per 128-token tile (zeroed together with the
 // accumulator), and the bf16 t x r result
-size_t lora_acc_bytes(int64_t t, int64_t r) { return align256(static_cast<size_t>(t) * r * 4); }
-size_t lora_counter_bytes(int64_t t) { return align256(static_cast<size_t>((t + 127) / 128) * 4); }
-size_t lora_region_bytes(int64_t t, int64_t r) {
-  return lora_acc_bytes(t, r) + lora_counter_bytes(t) + align256(static_cast<size_t>(t) * r * 2);
-}
+// workspace region of one rank-r down projection: t x r bf16 (sT or sU), 256-byte aligned
+size_t lora_region_bytes(int64_t t, int64_t r) { return align256(static_cast<size_t>(t) * r * 2); }
 
 // decode path (t <= 16): partial sums of X.L1 (gv::kDownParts x t x r fp32), the GEMV's fp32
 // t x o sums, its o / 32 tile counters
@@ -422,17 +419,12 @@ int launch_tc_gemm(const CUtensorMap& mA, const CUtensorMap& mB, int64_t M, int6
 }
 
 struct LoraWs {
-  float* acc32;        // t x r fp32
-  unsigned* counters;  // one per 128-token tile
-  uint16_t* b16;       // t x r bf16
+  uint16_t* b16;  // t x r bf16
 };
 
-LoraWs carve_lora(void* base, int64_t t, int64_t r) {
+LoraWs carve_lora(void* base, int64_t, int64_t) {
   LoraWs w;
-  uint8_t* b = reinterpret_cast<uint8_t*>(base);
-  w.acc32 = reinterpret_cast<float*>(b);
-  w.counters = reinterpret_cast<unsigned*>(b + lora_acc_bytes(t, r));
-  w.b16 = reinterpret_cast<uint16_t*>(b + lora_acc_bytes(t, r) + lora_counter_bytes(t));
+  w.b16 = reinterpret_cast<uint16_t*>(base);
   return w;
 }
 
