@@ -505,17 +505,42 @@ def main():
         hg = [(torch.empty(L.h, r, dtype=torch.float32).pin_memory(),
                torch.empty(r, L.o, dtype=torch.float32).pin_memory()) for L in layers]
 
+        # host->device copies on one stream, device->host on another, the linears on the
+        # compute stream: linear i+1's inputs cross the host link while linear i computes,
+        # and each linear's adapter gradients go back as soon as they exist
+        h2d_stream, d2h_stream = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        freed = [torch.cuda.Event() for _ in layers]   # compute is done with L.X, L.dY
+        for ev in freed:
+            ev.record()
+
         def e2e_step():
-            for L, x, dy, (g1, g2) in zip(layers, hX, hdY, hg):
-                L.X.copy_(x, non_blocking=True)
-                L.dY.copy_(dy, non_blocking=True)
+            comp = torch.cuda.current_stream(dev)
+            arrived = []
+            with torch.cuda.stream(h2d_stream):
+                for L, x, dy, fr in zip(layers, hX, hdY, freed):
+                    h2d_stream.wait_event(fr)
+                    L.X.copy_(x, non_blocking=True)
+                    L.dY.copy_(dy, non_blocking=True)
+                    ev = torch.cuda.Event()
+                    ev.record(h2d_stream)
+                    arrived.append(ev)
+            for L, ev, fr in zip(layers, arrived, freed):
+                comp.wait_event(ev)
                 L.step()
+                fr.record(comp)
             if world > 1:
                 from bit_quantized_lora_03_b200 import dp
                 dp.allreduce_adapter_grads([g for L in layers for g in (L.dL1, L.dL2)])
-            for L, (g1, g2) in zip(layers, hg):
-                g1.copy_(L.dL1, non_blocking=True)
-                g2.copy_(L.dL2, non_blocking=True)
+                reduced = torch.cuda.Event()
+                reduced.record(comp)
+            with torch.cuda.stream(d2h_stream):
+                for L, (g1, g2), fr in zip(layers, hg, freed):
+                    d2h_stream.wait_event(reduced if world > 1 else fr)
+                    g1.copy_(L.dL1, non_blocking=True)
+                    g2.copy_(L.dL2, non_blocking=True)
+                back = torch.cuda.Event()
+                back.record(d2h_stream)
+            comp.wait_event(back)   # a step ends when its gradients are on the host
         e2e_steps = max(3, args.steps // 2)
         e_ms = timed(e2e_step, e2e_steps, 1, world, dev)
         h2d = sum(x.numel() * 2 + dy.numel() * 2 for x, dy in zip(hX, hdY))

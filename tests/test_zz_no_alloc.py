@@ -53,7 +53,7 @@ def test_noalloc_matches_workspace_forward_twice(t, h, o, r, s):
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
     require_gpu()
-    t, h, o, r = 8192, 4096, 4096, 256       # needs 8192 * 256 * 6 bytes > 8 MiB
+    t, h, o, r = 32768, 1024, 1024, 256      # sT alone is 32768 * 256 * 2 bytes = 16 MiB > 8 MiB
     assert B.fwd_workspace_bytes(t, h, o, r) > B.QLORA_STATIC_SCRATCH_BYTES
     dev = torch.device("cuda")
     p = B.PackedNF4(o, h, dev)
