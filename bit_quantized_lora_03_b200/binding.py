@@ -45,6 +45,7 @@ SIGNATURES = {
     "qlora_get_last_status": (ctypes.c_int, [_PTR]),
     "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "qlora_set_gemv_max_ctas": (ctypes.c_int, [ctypes.c_int]),
+    "qlora_selftest_wait_timeout": (ctypes.c_int, [_I64, _PTR]),
     "qlora_profile_begin": (ctypes.c_int, [ctypes.c_int]),
     "qlora_profile_end": (ctypes.c_int, [_PTR, _PTR, ctypes.c_int]),
     "qlora_kernel_name": (ctypes.c_char_p, [ctypes.c_int]),
@@ -265,6 +266,12 @@ class KernelProfile:
             self.ms[name] = ms[k]
             self.launches[name] = n[k]
         return False
+
+
+def selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    """Launch the bounded-wait self-test (a wait nothing completes, given up after limit_ns)."""
+    _check(lib().qlora_selftest_wait_timeout(int(limit_ns), _stream(stream)),
+           "qlora_selftest_wait_timeout")
 
 
 def set_gemv_max_ctas(n: int) -> int:

@@ -69,17 +69,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase of `bar` with the given parity to complete. Returns false if the CTA's
-// abort flag is raised meanwhile, or if the wait exceeds kWaitTimeoutNs, in which case this
-// thread raises the abort flag and reports kDevTimeout. Never spins without bound.
+// abort flag is raised meanwhile, or if the wait exceeds limit_ns (kWaitTimeoutNs unless
+// given), in which case this thread raises the abort flag and reports kDevTimeout. Never spins
+// without bound.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          volatile uint32_t* abort_flag) {
+                                          volatile uint32_t* abort_flag,
+                                          uint64_t limit_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 15u) == 0u) {
       if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         *abort_flag = 1u;
         report(kDevTimeout);
         return false;

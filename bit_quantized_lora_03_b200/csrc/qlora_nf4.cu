@@ -496,6 +496,29 @@ int qlora_nf4_codebook(float* levels, float* midpoints) {
   return QLORA_OK;
 }
 
+// One thread waits on an mbarrier that no arrival will ever complete; the bounded wait gives
+// up after limit_ns, raises its CTA's abort flag and reports kDevTimeout. Nothing faults.
+__global__ void wait_timeout_selftest_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0u;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) (void)mbar_wait(&bar, 0u, &abort_flag, limit_ns);
+}
+
+int qlora_selftest_wait_timeout(int64_t limit_ns, qlora_stream_t stream) {
+  if (limit_ns < 1000 || limit_ns > static_cast<int64_t>(kWaitTimeoutNs)) return QLORA_ERR_INVALID_ARG;
+  int dev, rc;
+  if ((rc = current_device(&dev))) return rc;
+  wait_timeout_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(limit_ns));
+  return launch_status();
+}
+
 int qlora_set_gemv_max_ctas(int n) {
   return g_gemv_max_ctas.exchange(n > 0 ? n : 0);
 }

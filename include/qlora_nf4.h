@@ -206,6 +206,14 @@ QLORA_API const char *qlora_kernel_name(int kind);
  * previous cap (0 = none). Process-wide; not ordered with calls in flight on other threads. */
 QLORA_API int qlora_set_gemv_max_ctas(int n);
 
+/* Self-test of failure detection, with no counterpart in the method and no GPU fault: launches
+ * one kernel whose single thread waits on a barrier that nothing will complete, through the
+ * same bounded wait every pipelined kernel uses, with the limit shortened to limit_ns
+ * (1 us .. 2 s). When the limit passes, the wait gives up and QLORA_DEV_TIMEOUT is OR-ed into
+ * the status word, which qlora_get_last_status then returns; the context stays usable.
+ * Returns QLORA_ERR_INVALID_ARG for a limit outside that range. */
+QLORA_API int qlora_selftest_wait_timeout(int64_t limit_ns, qlora_stream_t stream);
+
 /* A static, human-readable name for any QLORA_* code (never NULL). */
 QLORA_API const char *qlora_status_string(int status);
 
