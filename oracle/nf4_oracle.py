@@ -383,6 +383,31 @@ def qlora_linear_bwd_dx_rows(rows, dY, Wdq, L1, L2, s):
     return dY @ Wt + s * ((dY @ L2.T) @ L1.T)
 
 
+# ----------------------------------------------------------------------------------------
+# Adapter merge ("QLoRA in LLMs" §11 "Saving, Loading, and Merging QLoRA Adapters": dequantize
+# the base into a wider precision, add the LoRA update, optionally quantize the result again,
+# and compare merged with unmerged outputs; "What it added up to", goodomens.studio: merging
+# into a 16-bit copy of the base changes the model the adapters compensated for)
+# ----------------------------------------------------------------------------------------
+
+def merge_adapters(Wdq, L1, L2, s):
+    """The merged weight in the stored orientation (o x h), fp64:
+    Wt_m[j][k] = Wdq[j][k] + s * sum_c L2[c][j] * L1[k][c], i.e. W_m = W' + s.L1.L2."""
+    Wt, L1, L2 = _f64(Wdq), _f64(L1), _f64(L2)
+    return Wt + s * (L2.T @ L1.T)
+
+
+def merge_error_bound(Wdq, L1, L2, s):
+    """Elementwise bound on |fp32 merge - merge_adapters| for an fp32 evaluation that sums the
+    r exact bf16 x bf16 products in any order (each partial sum rounded once), scales by s and
+    adds W' (two more roundings): (r + 2) * 2^-24 * (|W'| + |s| * sum_c |L2[c][j] L1[k][c]|),
+    doubled for margin."""
+    Wt, L1, L2 = _f64(Wdq), _f64(L1), _f64(L2)
+    r = L1.shape[1]
+    mag = np.abs(Wt) + abs(s) * (np.abs(L2).T @ np.abs(L1).T)
+    return 2.0 * (r + 2) * 2.0 ** -24 * mag
+
+
 def max_err_vs_rms(got, ref) -> tuple[float, float]:
     """(max |got - ref|, RMS(ref)) in fp64: the tolerance test is max <= 2e-2 * RMS."""
     got, ref = _f64(got), _f64(ref)
