@@ -46,6 +46,7 @@ SIGNATURES = {
     "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "qlora_set_gemv_max_ctas": (ctypes.c_int, [ctypes.c_int]),
     "qlora_selftest_wait_timeout": (ctypes.c_int, [_I64, _PTR]),
+    "qlora_merge_adapters": (ctypes.c_int, [_PTR, _PTR, _PTR, _I64, ctypes.c_float, _PTR, _PTR]),
     "qlora_profile_begin": (ctypes.c_int, [ctypes.c_int]),
     "qlora_profile_end": (ctypes.c_int, [_PTR, _PTR, ctypes.c_int]),
     "qlora_kernel_name": (ctypes.c_char_p, [ctypes.c_int]),
@@ -266,6 +267,23 @@ class KernelProfile:
             self.ms[name] = ms[k]
             self.launches[name] = n[k]
         return False
+
+
+def merge_adapters(p: PackedNF4, L1: torch.Tensor, L2: torch.Tensor, s: float,
+                   out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Wt_merged (o x h fp32) = W'^T + s.(L1.L2)^T: the adapters merged into the dequantized
+    base (re-quantize it with nf4_quantize for a merged packed weight)."""
+    o, h, r = p.out_features, p.in_features, L1.shape[1]
+    _require(L1, torch.bfloat16, (h, r), "L1")
+    _require(L2, torch.bfloat16, (r, o), "L2")
+    if out is None:
+        out = torch.empty(o, h, dtype=torch.float32, device=L1.device)
+    _require(out, torch.float32, (o, h), "out")
+    d = p.desc()
+    _check(lib().qlora_merge_adapters(ctypes.byref(d), L1.data_ptr(), L2.data_ptr(), r,
+                                      float(s), out.data_ptr(), _stream(stream)),
+           "qlora_merge_adapters")
+    return out
 
 
 def selftest_wait_timeout(limit_ns: int, stream=None) -> None:

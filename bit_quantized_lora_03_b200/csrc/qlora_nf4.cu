@@ -154,6 +154,9 @@ int current_device(int* dev_out) {
                                  static_cast<int>(gv::smem_bytes())) == cudaSuccess;
     fine &= cudaFuncSetAttribute(nf4_gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(gv::smem_bytes())) == cudaSuccess;
+    fine &= cudaFuncSetAttribute(tc_gemm_kernel<true, false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tcg::kMaxSmem) == cudaSuccess;
     fine &= cudaFuncSetAttribute(tc_gemm_kernel<false, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tcg::kMaxSmem) == cudaSuccess;
@@ -299,9 +302,6 @@ int check_linear_shape(int64_t t, int64_t h, int64_t o, int64_t r) {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// workspace region of one rank-r down projection (each part 256-byte aligned): the fp32
-// t x r split-K accumulator, one arrival counter per 128-token tile (zeroed together with the
-// accumulator), and the bf16 t x r result
 // workspace region of one rank-r down projection: t x r bf16 (sT or sU), 256-byte aligned
 size_t lora_region_bytes(int64_t t, int64_t r) { return align256(static_cast<size_t>(t) * r * 2); }
 
@@ -345,7 +345,7 @@ struct TcPlan {
 // per-CTA costs (set-up, epilogue, the final rounding) are paid as few times as possible.
 TcPlan plan_tc(int64_t M, int64_t ncols, int64_t K, bool b_mn, int sms) {
   TcPlan p{};
-  p.BNp = static_cast<int>((ncols + 15) / 16 * 16);
+  p.BNp = static_cast<int>(std::min<int64_t>(256, (ncols + 15) / 16 * 16));  // N > 256: N tiles
   p.num_kb = static_cast<int>((K + 63) / 64);
   p.mtiles = static_cast<int>((M + 127) / 128);
   int stages = tcg::MAX_STAGES;
@@ -376,7 +376,8 @@ TcPlan plan_tc(int64_t M, int64_t ncols, int64_t K, bool b_mn, int sms) {
 template <bool A_MN, bool B_MN>
 int launch_tc_gemm(const CUtensorMap& mA, const CUtensorMap& mB, int64_t M, int64_t ncols,
                    const TcPlan& pl, float alpha, int mode, float* out32, int64_t ld,
-                   uint16_t* o16a, uint16_t* o16b, int pdl, cudaStream_t st) {
+                   uint16_t* o16a, uint16_t* o16b, int pdl, cudaStream_t st,
+                   const nf4_weight* merge_w = nullptr) {
   TcGemmArgs a{};
   a.M = static_cast<int>(M);
   a.Ncols = static_cast<int>(ncols);
@@ -392,8 +393,15 @@ int launch_tc_gemm(const CUtensorMap& mA, const CUtensorMap& mB, int64_t M, int6
   a.out16a = o16a;
   a.out16b = o16b;
   a.pdl = pdl;
+  if (merge_w) {
+    a.codes = merge_w->codes;
+    a.q8 = merge_w->absmax_q8;
+    a.s2 = merge_w->absmax_s2;
+    a.tab = device_table();
+  }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(1, static_cast<unsigned>(pl.mtiles), static_cast<unsigned>(pl.splits));
+  cfg.gridDim = dim3(static_cast<unsigned>((ncols + pl.BNp - 1) / pl.BNp), static_cast<unsigned>(pl.mtiles),
+                     static_cast<unsigned>(pl.splits));
   cfg.blockDim = dim3(tcg::kThreads, 1, 1);
   cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = st;
@@ -494,6 +502,30 @@ int qlora_nf4_codebook(float* levels, float* midpoints) {
   std::memcpy(levels, cb.level, sizeof(cb.level));
   if (midpoints) std::memcpy(midpoints, cb.mid, sizeof(cb.mid));
   return QLORA_OK;
+}
+
+// W_m = W' + s.L1.L2 in the stored orientation ("QLoRA in LLMs" section 11: dequantize the
+// base into a wider precision and add the LoRA update): Wt_m (o x h fp32) = Wt' + s.L2^T.L1^T,
+// one tcgen05 product with K = r (A = L2 read MN-major, B = L1 read K-major, 128 x 256 output
+// tiles), the dequantized rows added in the epilogue.
+int qlora_merge_adapters(const nf4_weight* W, const uint16_t* L1, const uint16_t* L2, int64_t r,
+                         float s, float* Wt_merged, qlora_stream_t stream) {
+  if (!L1 || !L2 || !Wt_merged) return QLORA_ERR_INVALID_ARG;
+  if (!std::isfinite(s)) return QLORA_ERR_INVALID_ARG;
+  int rc = check_weight(W);
+  if (rc) return rc;
+  const int64_t h = W->in_features, o = W->out_features;
+  if ((rc = check_linear_shape(1, h, o, r))) return rc;
+  if (!aligned16(L1) || !aligned16(L2) || !aligned16(Wt_merged)) return QLORA_ERR_MISALIGNED;
+  int dev;
+  if ((rc = current_device(&dev))) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  CUtensorMap mA, mB;
+  const TcPlan pl = plan_tc(o, h, r, false, sm_count(dev));
+  if (!map_bf16(&mA, L2, o, r, 64, 64) || !map_bf16(&mB, L1, r, h, 64, static_cast<uint32_t>(pl.BNp)))
+    return QLORA_ERR_CUDA;
+  return launch_tc_gemm<true, false>(mA, mB, o, h, pl, s, kOutMergeNF4, Wt_merged, h, nullptr,
+                                     nullptr, kPdlNone, st, W);
 }
 
 // One thread waits on an mbarrier that no arrival will ever complete; the bounded wait gives

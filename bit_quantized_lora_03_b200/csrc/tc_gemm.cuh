@@ -40,6 +40,8 @@ enum TcOutMode : int {
   kOutRowMajor = 0,   // out32[m * ld + n] = acc (fp32)
   kOutTransposed = 1, // out32[n * ld + m] = acc (fp32)
   kOutRoundBf16 = 2,  // out16a[m * Ncols + n] = bf16(alpha * acc) (and out16b if set)
+  kOutMergeNF4 = 3,   // out32[m * ld + n] = W'[m][n] + alpha * acc, W' the dequantized NF4
+                      // row m (of ld = h weights) of the packed weight in the args
 };
 
 // Split-K runs as a thread-block cluster of `splits` CTAs along grid z (at most 8): each CTA
@@ -69,6 +71,11 @@ struct TcGemmArgs {
   uint16_t* out16a;
   uint16_t* out16b;
   int pdl;           // TcPdl
+  // kOutMergeNF4: the packed weight whose dequantized rows are added (Ncols = ld = h)
+  const uint8_t* codes;
+  const uint8_t* q8;
+  const float* s2;
+  Nf4Table tab;
 };
 
 #ifdef QLORA_TRACE
@@ -102,6 +109,7 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.y * BM;
+  const int nb0 = blockIdx.x * BNp;  // this CTA's first output column (N tiles along grid x)
   const int kb0 = blockIdx.z * args.kb_per_split;
   const int kb1 = min(args.num_kb, kb0 + args.kb_per_split);
   const int nk = kb1 - kb0;
@@ -109,6 +117,8 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
   const int b_atoms = (BNp + 63) / 64;
   const uint32_t bbytes = static_cast<uint32_t>(b_bytes(BNp, B_MN));
   pdl_launch_dependents();
+  __shared__ float mlv[16];  // NF4 levels (kOutMergeNF4)
+  if (threadIdx.x < 16) mlv[threadIdx.x] = args.tab.level[threadIdx.x];
 
   if (threadIdx.x == 0) {
     QLORA_STAMP(0);
@@ -153,10 +163,10 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
         }
         uint8_t* b_dst = a_dst + A_BYTES;
         if (!B_MN) {
-          tma_load_2d(b_dst, &tmB, &full[slot], kb * BK, 0);
+          tma_load_2d(b_dst, &tmB, &full[slot], kb * BK, nb0);
         } else {
           for (int a = 0; a < b_atoms; ++a)
-            tma_load_2d(b_dst + a * 8192, &tmB, &full[slot], a * 64, kb * BK);
+            tma_load_2d(b_dst + a * 8192, &tmB, &full[slot], nb0 + a * 64, kb * BK);
         }
         if (i == 0) QLORA_STAMP(2);
         issued = i + 1;
@@ -214,8 +224,28 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
                           __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
         return;
       }
+      n0 += nb0;
       if (row >= args.M || n0 >= args.Ncols) return;
-      if (args.out_mode == kOutTransposed) {
+      if (args.out_mode == kOutMergeNF4) {
+        // the 16 dequantized weights W'[row][n0 .. n0+15]: 8 code bytes, one 8-bit scale
+        const int64_t e0 = static_cast<int64_t>(row) * args.ld + n0;
+        const uint2 cw = *reinterpret_cast<const uint2*>(args.codes + e0 / 2);
+        const int64_t blk = e0 / kBlock;
+        const float k = __fmul_rn(static_cast<float>(args.q8[blk]), args.s2[blk / kGroup]);
+        float* dst = args.out32 + e0;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint32_t w2 = (q4 < 2 ? cw.x : cw.y) >> (16 * (q4 & 1));   // bytes 2 q4, 2 q4 + 1
+          float o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t code = (w2 >> ((e >> 1) * 8 + ((e & 1) ? 0 : 4))) & 15u;
+            const float wq = __bfloat162float(__float2bfloat16_rn(__fmul_rn(mlv[code], k)));
+            o[e] = __fadd_rn(wq, __fmul_rn(args.alpha, __uint_as_float(v[4 * q4 + e])));
+          }
+          *reinterpret_cast<float4*>(dst + 4 * q4) = make_float4(o[0], o[1], o[2], o[3]);
+        }
+      } else if (args.out_mode == kOutTransposed) {
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           args.out32[static_cast<int64_t>(n0 + e) * args.ld + row] = __uint_as_float(v[e]);
@@ -282,17 +312,19 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
     const int r0 = q * BM / S, r1 = (q + 1) * BM / S, nr = r1 - r0;
     const float* part0 = reinterpret_cast<const float*>(smem);
     const int ld_s = BNp + 4;
+    const int tile_cols = args.Ncols - nb0 < BNp ? args.Ncols - nb0 : BNp;
     if (!*abort_flag) {
       if (args.out_mode == kOutTransposed) {
         // consecutive threads take consecutive rows of one column: coalesced column stores
-        for (int e = threadIdx.x; e < nr * args.Ncols; e += kThreads) {
+        for (int e = threadIdx.x; e < nr * tile_cols; e += kThreads) {
           const int rl = r0 + e % nr, n = e / nr;
           float sum = 0.f;
           for (int p = 0; p < S; ++p) sum += ld_dsmem_f32(part0 + rl * ld_s + n, static_cast<uint32_t>(p));
-          if (m0 + rl < args.M) args.out32[static_cast<int64_t>(n) * args.ld + m0 + rl] = sum;
+          if (m0 + rl < args.M && nb0 + n < args.Ncols)
+            args.out32[static_cast<int64_t>(nb0 + n) * args.ld + m0 + rl] = sum;
         }
       } else {
-        const int nq = args.Ncols / 4;
+        const int nq = tile_cols / 4;
         for (int e = threadIdx.x; e < nr * nq; e += kThreads) {
           const int rl = r0 + e / nq, n = 4 * (e % nq);
           float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -300,17 +332,17 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
             const float4 v = ld_dsmem_f32x4(part0 + rl * ld_s + n, static_cast<uint32_t>(p));
             sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
           }
-          if (m0 + rl >= args.M) continue;
+          if (m0 + rl >= args.M || nb0 + n >= args.Ncols) continue;
           if (args.out_mode == kOutRoundBf16) {
             const float a = args.alpha;
             uint2 o;
             o.x = pack_bf16x2(a * sum.x, a * sum.y);
             o.y = pack_bf16x2(a * sum.z, a * sum.w);
-            const int64_t off = static_cast<int64_t>(m0 + rl) * args.Ncols + n;
+            const int64_t off = static_cast<int64_t>(m0 + rl) * args.Ncols + nb0 + n;
             *reinterpret_cast<uint2*>(args.out16a + off) = o;
             if (args.out16b) *reinterpret_cast<uint2*>(args.out16b + off) = o;
           } else {
-            *reinterpret_cast<float4*>(args.out32 + static_cast<int64_t>(m0 + rl) * args.ld + n) = sum;
+            *reinterpret_cast<float4*>(args.out32 + static_cast<int64_t>(m0 + rl) * args.ld + nb0 + n) = sum;
           }
         }
       }

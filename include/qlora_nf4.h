@@ -198,6 +198,22 @@ QLORA_API int qlora_profile_begin(int capacity);
 QLORA_API int qlora_profile_end(double *ms, int64_t *launches, int nkinds);
 QLORA_API const char *qlora_kernel_name(int kind);
 
+/* Adapter merge ("QLoRA in LLMs" section 11, "Saving, Loading, and Merging QLoRA Adapters":
+ * dequantize the base into a wider precision, add the LoRA update, optionally quantize the
+ * result again): Wt_merged = W'^T + s . (L1 . L2)^T, i.e. W_m = W' + s.L1.L2 in the stored
+ * orientation, in fp32:
+ *   Wt_merged[j][k] = W'[k][j] + s * sum_c L1[k][c] * L2[c][j]    (o x h, row-major)
+ * where W'[k][j] is the nf4_dequantize value (exact bf16) of the packed weight. The rank-r
+ * sum is formed from the exact bf16 products in fp32; each element is within
+ * (r + 2) * 2^-23 * (|W'| + |s| * sum_c |L1 L2|) of the exact merge. Re-quantize the result
+ * with nf4_quantize to obtain a merged packed weight.
+ *   W: packed weight (out_features o, in_features h: h % 64 == 0, o % 64 == 0).
+ *   L1 (h x r), L2 (r x o): bf16 row-major, 16 <= r <= 256, r % 16 == 0.
+ *   Wt_merged: caller-owned device buffer of o * h fp32, 16-byte aligned; overwritten.
+ * Errors: QLORA_ERR_INVALID_ARG / _BAD_SHAPE / _MISALIGNED / _CUDA, nothing launched. */
+QLORA_API int qlora_merge_adapters(const nf4_weight *W, const uint16_t *L1, const uint16_t *L2,
+                                   int64_t r, float s, float *Wt_merged, qlora_stream_t stream);
+
 /* Launch shape of the decode GEMV (t <= 16), a scheduling knob with no counterpart in the
  * method. By default the GEMV runs one CTA of 16 warps per SM and splits its units (32 rows x
  * 128 inputs) evenly over all their warps. qlora_set_gemv_max_ctas(n) caps that CTA count at
