@@ -375,6 +375,58 @@ def stack65b_leg(dev, peaks, steps: int = 2, warmup: int = 1):
     return res
 
 
+def merge_leg(dev, peaks, r: int = 64, s: float = 0.25):
+    """Adapter merge over the 7 linears of the LLaMA-7B-shaped layer: GB/s of the merge
+    (write 4 B + read 0.516 B per weight) and of the re-quantization, and the output drift of
+    one linear (up_proj, 4096 tokens) merged two ways against the unmerged layer: into the
+    dequantized base then re-quantized to NF4, and into a 16-bit copy of the original base."""
+    from bit_quantized_lora_03_b200 import binding as B
+    from bit_quantized_lora_03_b200 import inputs
+    lins = [inputs.training_linear(i, r=r, s=s) for i in range(7)]
+    packs = [B.nf4_quantize(li.Wt.to(dev)) for li in lins]
+    L1s = [li.L1.to(dev) for li in lins]
+    L2s = [li.L2.to(dev) for li in lins]
+    outs = [torch.empty(li.o, li.h, dtype=torch.float32, device=dev) for li in lins]
+    reqs = [B.PackedNF4(li.o, li.h, dev) for li in lins]
+    n = sum(li.o * li.h for li in lins)
+
+    def merge():
+        for p, a, b, o_ in zip(packs, L1s, L2s, outs):
+            B.merge_adapters(p, a, b, s, out=o_)
+
+    def requant():
+        for o_, q in zip(outs, reqs):
+            B.nf4_quantize(o_, out=q)
+    mms = queued_ms(merge, 5, 2) / 5
+    qms = queued_ms(requant, 5, 2) / 5
+    mbytes = 4 * n + sum(p.nbytes for p in packs) + sum(2 * (a.numel() + b.numel()) for a, b in zip(L1s, L2s))
+    # drift of up_proj
+    li, p, pm = lins[5], packs[5], reqs[5]
+    X = li.X.to(dev)
+    Yu, _ = B.qlora_linear_fwd(X, p, L1s[5], L2s[5], s, want_sT=False)
+    zero1, zero2 = torch.zeros_like(L1s[5]), torch.zeros_like(L2s[5])
+    Ym, _ = B.qlora_linear_fwd(X, pm, zero1, zero2, 0.0, want_sT=False)
+    W16 = (li.Wt.to(dev) + s * (L1s[5].float() @ L2s[5].float()).t()).to(torch.bfloat16)
+    Y16 = X @ W16.t()   # a plain bf16 library GEMM, for the report only
+    torch.cuda.synchronize()
+
+    def rel(a, b):
+        return round(float((a.float() - b.float()).pow(2).mean().sqrt() / b.float().pow(2).mean().sqrt()), 5)
+    res = {
+        "weights": n, "r": r, "s": s,
+        "merge_ms": round(mms, 4), "merge_gbs": round(mbytes / (mms * 1e-3) / 1e9, 1),
+        "merge_frac_hbm": round(mbytes / (mms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
+        "requantize_ms": round(qms, 4),
+        "drift_up_proj_t4096": {
+            "merged_into_dequantized_then_nf4_vs_unmerged_rel_rms": rel(Ym, Yu),
+            "merged_into_16bit_original_vs_unmerged_rel_rms": rel(Y16, Yu)},
+        "device_status": B.last_status(),
+    }
+    del packs, outs, reqs, L1s, L2s
+    torch.cuda.empty_cache()
+    return res
+
+
 # ------------------------------------------------------------------------------------------
 # CPU oracle baseline (bounded sample)
 # ------------------------------------------------------------------------------------------
@@ -577,6 +629,7 @@ def main():
         legs["decode_gemv"] = gemv_leg(dev, peaks, l2_bytes)
         legs["codec_llama7b_layer"] = codec_leg(dev, peaks)
         legs["stack65b"] = stack65b_leg(dev, peaks)
+        legs["merge_llama7b_layer"] = merge_leg(dev, peaks)
         tps, sec, _ = oracle_sample(args.cpu_sample_tokens)
         cpu = {"value": round(tps, 3), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                "sample": (f"fwd+bwd of {args.cpu_sample_tokens} of the 4096 tokens, one linear per "
