@@ -370,6 +370,11 @@ TcPlan plan_tc(int64_t M, int64_t ncols, int64_t K, bool b_mn, int sms) {
     splits = 1;
   p.kb_per_split = (p.num_kb + splits - 1) / splits;
   p.splits = (p.num_kb + p.kb_per_split - 1) / p.kb_per_split;
+  // no more stages than K-steps per CTA (a short K leaves room for more CTAs per SM)
+  if (p.stages > std::max(2, p.kb_per_split)) {
+    p.stages = std::max(2, p.kb_per_split);
+    p.smem = tcg::smem_bytes(p.stages, p.BNp, b_mn);
+  }
   return p;
 }
 

@@ -226,26 +226,7 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
       }
       n0 += nb0;
       if (row >= args.M || n0 >= args.Ncols) return;
-      if (args.out_mode == kOutMergeNF4) {
-        // the 16 dequantized weights W'[row][n0 .. n0+15]: 8 code bytes, one 8-bit scale
-        const int64_t e0 = static_cast<int64_t>(row) * args.ld + n0;
-        const uint2 cw = *reinterpret_cast<const uint2*>(args.codes + e0 / 2);
-        const int64_t blk = e0 / kBlock;
-        const float k = __fmul_rn(static_cast<float>(args.q8[blk]), args.s2[blk / kGroup]);
-        float* dst = args.out32 + e0;
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const uint32_t w2 = (q4 < 2 ? cw.x : cw.y) >> (16 * (q4 & 1));   // bytes 2 q4, 2 q4 + 1
-          float o[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t code = (w2 >> ((e >> 1) * 8 + ((e & 1) ? 0 : 4))) & 15u;
-            const float wq = __bfloat162float(__float2bfloat16_rn(__fmul_rn(mlv[code], k)));
-            o[e] = __fadd_rn(wq, __fmul_rn(args.alpha, __uint_as_float(v[4 * q4 + e])));
-          }
-          *reinterpret_cast<float4*>(dst + 4 * q4) = make_float4(o[0], o[1], o[2], o[3]);
-        }
-      } else if (args.out_mode == kOutTransposed) {
+      if (args.out_mode == kOutTransposed) {
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           args.out32[static_cast<int64_t>(n0 + e) * args.ld + row] = __uint_as_float(v[e]);
@@ -277,7 +258,55 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
       }
     };
     const int nchunks = BNp / 16;
-    if (ok && !*abort_flag) {
+    if (ok && !*abort_flag && args.out_mode == kOutMergeNF4 && args.splits == 1) {
+      // 64 columns (one NF4 block of this row) per round: the next block's 32 code bytes and
+      // scales are loaded while this one's accumulator chunks come out of TMEM
+      const int64_t rowbase = static_cast<int64_t>(row) * args.ld;
+      const bool rok = row < args.M;
+      auto load_block = [&](int col, uint4& ca, uint4& cb, float& k) {
+        if (rok && col < args.Ncols) {
+          const uint4* src = reinterpret_cast<const uint4*>(args.codes + (rowbase + col) / 2);
+          ca = src[0];
+          cb = src[1];
+          const int64_t blk = (rowbase + col) / kBlock;
+          k = __fmul_rn(static_cast<float>(args.q8[blk]), args.s2[blk / kGroup]);
+        }
+      };
+      uint4 ca = make_uint4(0u, 0u, 0u, 0u), cb = ca;
+      float kk = 0.f;
+      load_block(nb0, ca, cb, kk);
+      for (int c = 0; c < nchunks; c += 4) {
+        uint32_t v[4][16];
+        tmem_ld_16(lane_addr + c * 16, v[0]);
+        tmem_ld_16(lane_addr + (c + 1) * 16, v[1]);
+        tmem_ld_16(lane_addr + (c + 2) * 16, v[2]);
+        tmem_ld_16(lane_addr + (c + 3) * 16, v[3]);
+        uint4 na = ca, nbk = cb;
+        float nk = kk;
+        if (c + 4 < nchunks) load_block(nb0 + (c + 4) * 16, na, nbk, nk);
+        tmem_ld_wait();
+        const int col0 = nb0 + c * 16;
+        if (rok && col0 < args.Ncols) {
+          const uint32_t words[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+          float* dst = args.out32 + rowbase + col0;
+#pragma unroll
+          for (int w = 0; w < 8; ++w) {          // 8 weights per code word
+            float o[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {        // element 2j: high nibble of byte j
+              const uint32_t code = (words[w] >> ((e >> 1) * 8 + ((e & 1) ? 0 : 4))) & 15u;
+              const float wq = __bfloat162float(__float2bfloat16_rn(__fmul_rn(mlv[code], kk)));
+              o[e] = __fadd_rn(wq, __fmul_rn(args.alpha, __uint_as_float(v[w >> 1][(w & 1) * 8 + e])));
+            }
+            *reinterpret_cast<float4*>(dst + 8 * w) = make_float4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<float4*>(dst + 8 * w + 4) = make_float4(o[4], o[5], o[6], o[7]);
+          }
+        }
+        ca = na;
+        cb = nbk;
+        kk = nk;
+      }
+    } else if (ok && !*abort_flag) {
       // up to four 16-column TMEM loads in flight before one wait (the counts are warp-uniform)
       for (int c = 0; c < nchunks; c += 4) {
         uint32_t v0[16], v1[16], v2[16], v3[16];
