@@ -206,11 +206,12 @@ def block_absmax(Wt: np.ndarray) -> np.ndarray:
     return np.max(np.abs(w), axis=1)
 
 
-def nf4_codes(Wt: np.ndarray, levels: np.ndarray | None = None) -> np.ndarray:
+def nf4_codes(Wt: np.ndarray, levels: np.ndarray | None = None,
+              zero_code: int = ZERO_CODE) -> np.ndarray:
     """Unpacked 4-bit codes (uint8, one per weight) from the exact fp32 block absmax.
 
     x_hat = w / c1 in fp32 (IEEE, round to nearest); code = number of midpoints strictly
-    below x_hat. A block whose absmax is 0 takes the zero level everywhere.
+    below x_hat. A block whose absmax is 0 takes the zero level (code `zero_code`) everywhere.
     """
     mid = nf4_midpoints(levels)
     w = np.asarray(Wt, dtype=np.float32).reshape(-1, BLOCK)
@@ -221,7 +222,7 @@ def nf4_codes(Wt: np.ndarray, levels: np.ndarray | None = None) -> np.ndarray:
     codes = np.zeros(w.shape, dtype=np.uint8)
     for i in range(mid.size):
         codes += (xhat > mid[i]).astype(np.uint8)
-    codes[zero, :] = ZERO_CODE
+    codes[zero, :] = zero_code
     return codes.reshape(-1)
 
 
@@ -278,6 +279,55 @@ def nf4_quantize(Wt: np.ndarray) -> NF4Packed:
     codes = nf4_codes(Wt)
     q8, s2 = double_quantize(c1)
     return NF4Packed(pack_nibbles(codes), q8, s2, Wt.shape[0], Wt.shape[1], c1)
+
+
+# ----------------------------------------------------------------------------------------
+# Other 4-bit codebooks, for the format comparison the pages draw (NF4 against FP4 and INT4:
+# "QLoRA in LLMs" §5 and "Idea one: NF4", goodomens.studio; the textbook absmax integer scheme
+# of "QLoRA in LLMs" §2). Same blocks, packing and double-quantized scales; only the 16 levels
+# (and the code of the zero level, used for all-zero blocks) differ.
+# ----------------------------------------------------------------------------------------
+
+def fp4_codebook() -> np.ndarray:
+    """FP4 E2M1: magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6} with both signs, divided by the
+    largest (6) so the ends are -1 and +1; -0 and +0 are both kept (16 codes), ascending."""
+    mags = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    neg = [-m / 6.0 for m in reversed(mags)]      # -1 ... -0
+    pos = [m / 6.0 for m in mags]                 # +0 ... +1
+    return np.array(neg + pos, dtype=np.float64).astype(np.float32)
+
+
+def int4_codebook() -> np.ndarray:
+    """Symmetric absmax INT4: k / 7 for k = -8 .. 7 (the textbook absmax scheme with 4-bit
+    integers; k = -8 lies below -1 and is never the nearest level of an |x| <= 1)."""
+    return np.array([k / 7.0 for k in range(-8, 8)], dtype=np.float64).astype(np.float32)
+
+
+# codebook id (the ids of the library's codebook calls) -> code of its zero level
+CODEBOOK_ZERO_CODE = {0: ZERO_CODE, 1: 7, 2: 8}
+
+
+def codebook_levels(cb: int) -> np.ndarray:
+    return {0: nf4_codebook, 1: fp4_codebook, 2: int4_codebook}[cb]()
+
+
+def quantize_with(Wt: np.ndarray, cb: int) -> NF4Packed:
+    """nf4_quantize with codebook `cb` (0 NF4, 1 FP4, 2 INT4): same blocks, packing and
+    double quantization; codes from that codebook's midpoints."""
+    Wt = np.asarray(Wt, dtype=np.float32)
+    if Wt.ndim != 2 or Wt.shape[1] % BLOCK != 0:
+        raise ValueError("Wt must be o x h with h a multiple of 64")
+    if not np.all(np.isfinite(Wt)):
+        raise ValueError("non-finite weight")
+    c1 = block_absmax(Wt)
+    codes = nf4_codes(Wt, codebook_levels(cb), CODEBOOK_ZERO_CODE[cb])
+    q8, s2 = double_quantize(c1)
+    return NF4Packed(pack_nibbles(codes), q8, s2, Wt.shape[0], Wt.shape[1], c1)
+
+
+def dequantize_bits_with(packed: NF4Packed, cb: int) -> np.ndarray:
+    """bf16 bit patterns of bf16(level[code] * (q8 * s2)) with codebook `cb`."""
+    return bf16_bits_rne(nf4_dequantize_f32(packed, codebook_levels(cb)))
 
 
 def block_scales(q8: np.ndarray, s2: np.ndarray) -> np.ndarray:
