@@ -47,6 +47,9 @@ SIGNATURES = {
     "qlora_set_gemv_max_ctas": (ctypes.c_int, [ctypes.c_int]),
     "qlora_selftest_wait_timeout": (ctypes.c_int, [_I64, _PTR]),
     "qlora_merge_adapters": (ctypes.c_int, [_PTR, _PTR, _PTR, _I64, ctypes.c_float, _PTR, _PTR]),
+    "qlora_codebook": (ctypes.c_int, [ctypes.c_int, _PTR, _PTR]),
+    "qlora_quantize_codebook": (ctypes.c_int, [_PTR, _PTR, ctypes.c_int, _PTR]),
+    "qlora_dequantize_codebook": (ctypes.c_int, [_PTR, ctypes.c_int, _PTR, _PTR]),
     "qlora_profile_begin": (ctypes.c_int, [ctypes.c_int]),
     "qlora_profile_end": (ctypes.c_int, [_PTR, _PTR, ctypes.c_int]),
     "qlora_kernel_name": (ctypes.c_char_p, [ctypes.c_int]),
@@ -106,11 +109,19 @@ def _ptr(t: torch.Tensor | None) -> int | None:
     return None if t is None else t.data_ptr()
 
 
-def codebook():
-    """(levels[16], midpoints[15]) as derived by the library (host call, no GPU needed)."""
+CODEBOOK_NF4, CODEBOOK_FP4, CODEBOOK_INT4 = 0, 1, 2
+
+
+def codebook(codebook_id: int | None = None):
+    """(levels[16], midpoints[15]) as derived by the library (host call, no GPU needed);
+    the NF4 codebook unless another id is given."""
     lv = (ctypes.c_float * 16)()
     md = (ctypes.c_float * 15)()
-    _check(lib().qlora_nf4_codebook(ctypes.cast(lv, _PTR), ctypes.cast(md, _PTR)), "codebook")
+    if codebook_id is None:
+        _check(lib().qlora_nf4_codebook(ctypes.cast(lv, _PTR), ctypes.cast(md, _PTR)), "codebook")
+    else:
+        _check(lib().qlora_codebook(int(codebook_id), ctypes.cast(lv, _PTR), ctypes.cast(md, _PTR)),
+               "codebook")
     return list(lv), list(md)
 
 
@@ -142,25 +153,37 @@ def _require(t: torch.Tensor, dtype, shape, name: str) -> None:
                          f"got {t.dtype} {tuple(t.shape)} on {t.device}")
 
 
-def nf4_quantize(Wt: torch.Tensor, out: PackedNF4 | None = None, stream=None) -> PackedNF4:
-    """Quantize an fp32 CUDA weight Wt (o x h) to packed NF4 with double-quantized scales."""
+def nf4_quantize(Wt: torch.Tensor, out: PackedNF4 | None = None, stream=None,
+                 codebook_id: int = CODEBOOK_NF4) -> PackedNF4:
+    """Quantize an fp32 CUDA weight Wt (o x h) to packed 4-bit codes with double-quantized
+    scales (NF4 unless another codebook id is given)."""
     o, h = Wt.shape
     _require(Wt, torch.float32, (o, h), "Wt")
     p = out if out is not None else PackedNF4(o, h, Wt.device)
     d = p.desc()
-    _check(lib().nf4_quantize(Wt.data_ptr(), ctypes.byref(d), _stream(stream)), "nf4_quantize")
+    if codebook_id == CODEBOOK_NF4:
+        _check(lib().nf4_quantize(Wt.data_ptr(), ctypes.byref(d), _stream(stream)), "nf4_quantize")
+    else:
+        _check(lib().qlora_quantize_codebook(Wt.data_ptr(), ctypes.byref(d), int(codebook_id),
+                                             _stream(stream)), "qlora_quantize_codebook")
     return p
 
 
-def nf4_dequantize(p: PackedNF4, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """The bf16 weight Wt' (o x h) reconstructed from a packed weight."""
+def nf4_dequantize(p: PackedNF4, out: torch.Tensor | None = None, stream=None,
+                   codebook_id: int = CODEBOOK_NF4) -> torch.Tensor:
+    """The bf16 weight Wt' (o x h) reconstructed from a packed weight (with the codebook it
+    was packed with)."""
     if out is None:
         out = torch.empty(p.out_features, p.in_features, dtype=torch.bfloat16,
                           device=p.codes.device)
     _require(out, torch.bfloat16, (p.out_features, p.in_features), "out")
     d = p.desc()
-    _check(lib().nf4_dequantize(ctypes.byref(d), out.data_ptr(), _stream(stream)),
-           "nf4_dequantize")
+    if codebook_id == CODEBOOK_NF4:
+        _check(lib().nf4_dequantize(ctypes.byref(d), out.data_ptr(), _stream(stream)),
+               "nf4_dequantize")
+    else:
+        _check(lib().qlora_dequantize_codebook(ctypes.byref(d), int(codebook_id), out.data_ptr(),
+                                               _stream(stream)), "qlora_dequantize_codebook")
     return out
 
 

@@ -17,6 +17,7 @@ namespace qlora {
 struct Nf4Table {
   float level[16];
   float mid[16];  // 15 thresholds, mid[15] unused
+  int zero_code;  // code of the zero level (all-zero blocks): 7 for NF4
 };
 
 constexpr int kBlock = 64;
@@ -24,8 +25,9 @@ constexpr int kGroup = 256;
 
 // Nearest-level code of x = w / c1 as the number of thresholds strictly below x, found by a
 // four-step binary search over the sorted thresholds in shared memory.
-__device__ __forceinline__ uint32_t nf4_code_of(float w, float c1, const float* mids) {
-  if (c1 == 0.0f) return 7u;
+__device__ __forceinline__ uint32_t nf4_code_of(float w, float c1, const float* mids,
+                                                uint32_t zero_code = 7u) {
+  if (c1 == 0.0f) return zero_code;
   const float x = __fdiv_rn(w, c1);
   uint32_t c = (x > mids[7]) ? 8u : 0u;
   c += (x > mids[c + 3]) ? 4u : 0u;
@@ -50,8 +52,9 @@ struct Nf4Buckets {
   int exact_only;
 };
 
-__device__ __noinline__ uint32_t nf4_code_exact(float w, float c1, const float* mids) {
-  return nf4_code_of(w, c1, mids);
+__device__ __noinline__ uint32_t nf4_code_exact(float w, float c1, const float* mids,
+                                               uint32_t zero_code) {
+  return nf4_code_of(w, c1, mids, zero_code);
 }
 
 // Fast decision; sets `near` when x' is within 2^-20 of the bucket's threshold (the caller
@@ -103,6 +106,7 @@ __global__ void __launch_bounds__(qz::kThreads, 1) nf4_quantize_kernel(
   for (int i = tid; i < 128 * 32; i += qz::kThreads)
     bk[i] = make_float2(bkt.thr[i >> 5], __uint_as_float(static_cast<uint32_t>(bkt.lo[i >> 5])));
   const bool fast = bkt.exact_only == 0;
+  const uint32_t zc = static_cast<uint32_t>(tab.zero_code);
   const uint32_t lane_tab = smem_addr(bk) + static_cast<uint32_t>(tid & 31) * 8u;
   const int h32 = tid >> 4, l16 = tid & 15;
   const int64_t ngroups = (nblocks + kGroup - 1) / kGroup;
@@ -159,10 +163,10 @@ __global__ void __launch_bounds__(qz::kThreads, 1) nf4_quantize_kernel(
           k3 = nf4_code_fast(x.w, rc, lane_tab, near);
         }
         if (near) {  // rare: some weight lies next to a threshold, or c1 is tiny
-          k0 = nf4_code_exact(x.x, a, mids);
-          k1 = nf4_code_exact(x.y, a, mids);
-          k2 = nf4_code_exact(x.z, a, mids);
-          k3 = nf4_code_exact(x.w, a, mids);
+          k0 = nf4_code_exact(x.x, a, mids, zc);
+          k1 = nf4_code_exact(x.y, a, mids, zc);
+          k2 = nf4_code_exact(x.z, a, mids, zc);
+          k3 = nf4_code_exact(x.w, a, mids, zc);
         }
         const uint32_t packed = ((k0 << 4) | k1) | (((k2 << 4) | k3) << 8);
         *reinterpret_cast<uint16_t*>(codes + g * (kGroup * kBlock / 2) + blk * 32 + l16 * 2) =

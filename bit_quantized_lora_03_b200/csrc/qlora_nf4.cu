@@ -55,41 +55,71 @@ double normal_quantile(double p) {
 struct Codebook {
   float level[16];
   float mid[15];
+  int zero_code;  // the code of the zero level (all-zero blocks)
 };
 
-const Codebook& codebook() {
-  static Codebook cb = [] {
-    Codebook c{};
-    const double delta = 0.5 * ((1.0 - 1.0 / 30.0) + (1.0 - 1.0 / 32.0));
-    std::vector<double> v;
-    for (int i = 0; i < 8; ++i) v.push_back(normal_quantile(delta + i * (0.5 - delta) / 8.0));
-    for (int i = 0; i < 7; ++i) v.push_back(-normal_quantile(delta + i * (0.5 - delta) / 7.0));
-    v.push_back(0.0);
-    std::sort(v.begin(), v.end());
-    const double top = normal_quantile(delta);
-    for (int i = 0; i < 16; ++i) c.level[i] = static_cast<float>(v[i] / top);
-    for (int i = 0; i < 15; ++i)
-      c.mid[i] = static_cast<float>((static_cast<double>(c.level[i]) +
-                                     static_cast<double>(c.level[i + 1])) / 2.0);
-    return c;
-  }();
-  return cb;
+Codebook finish(const double (&v)[16], int zero_code) {
+  Codebook c{};
+  for (int i = 0; i < 16; ++i) c.level[i] = static_cast<float>(v[i]);
+  for (int i = 0; i < 15; ++i)
+    c.mid[i] = static_cast<float>((static_cast<double>(c.level[i]) +
+                                   static_cast<double>(c.level[i + 1])) / 2.0);
+  c.zero_code = zero_code;
+  return c;
 }
 
-Nf4Table device_table() {
+// Codebook ids: 0 NF4 (above); 1 FP4 E2M1, magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6} with both
+// signs over 6 (both zeros kept); 2 absmax INT4, k / 7 for k = -8 .. 7 (the textbook absmax
+// integer scheme, "QLoRA in LLMs" section 2). Same blocks, packing and scales; the pages set
+// NF4 against these two ("QLoRA in LLMs" section 5; "Idea one: NF4", goodomens.studio).
+constexpr int kCodebooks = 3;
+
+const Codebook& codebook(int id = 0) {
+  static const Codebook cbs[kCodebooks] = {
+      [] {
+        const double delta = 0.5 * ((1.0 - 1.0 / 30.0) + (1.0 - 1.0 / 32.0));
+        std::vector<double> v;
+        for (int i = 0; i < 8; ++i) v.push_back(normal_quantile(delta + i * (0.5 - delta) / 8.0));
+        for (int i = 0; i < 7; ++i) v.push_back(-normal_quantile(delta + i * (0.5 - delta) / 7.0));
+        v.push_back(0.0);
+        std::sort(v.begin(), v.end());
+        const double top = normal_quantile(delta);
+        double w[16];
+        for (int i = 0; i < 16; ++i) w[i] = v[i] / top;
+        return finish(w, 7);
+      }(),
+      [] {
+        const double mags[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+        double w[16];
+        for (int i = 0; i < 8; ++i) {
+          w[i] = -mags[7 - i] / 6.0;  // -1 ... -0
+          w[8 + i] = mags[i] / 6.0;   // +0 ... +1
+        }
+        return finish(w, 7);
+      }(),
+      [] {
+        double w[16];
+        for (int k = -8; k < 8; ++k) w[k + 8] = k / 7.0;
+        return finish(w, 8);
+      }()};
+  return cbs[id];
+}
+
+Nf4Table device_table(int id = 0) {
   Nf4Table t{};
-  const Codebook& cb = codebook();
+  const Codebook& cb = codebook(id);
   for (int i = 0; i < 16; ++i) t.level[i] = cb.level[i];
   for (int i = 0; i < 15; ++i) t.mid[i] = cb.mid[i];
   t.mid[15] = 2.0f;
+  t.zero_code = cb.zero_code;
   return t;
 }
 
 // Buckets of the quantizer's fast decision (see nf4_code_fast): bucket b covers
 // [-1 + b/64, -1 + (b+1)/64); fp32 arithmetic on these edges is exact.
-Nf4Buckets device_buckets() {
+Nf4Buckets device_buckets(int id = 0) {
   Nf4Buckets bk{};
-  const Codebook& cb = codebook();
+  const Codebook& cb = codebook(id);
   int bad = 0;
   for (int b = 0; b < 128; ++b) {
     const float lo = -1.0f + static_cast<float>(b) / 64.0f, hi = lo + 1.0f / 64.0f;
@@ -658,8 +688,10 @@ int qlora_get_last_status(qlora_stream_t stream) {
   return static_cast<int>(v);
 }
 
-int nf4_quantize(const float* Wt, const nf4_weight* q, qlora_stream_t stream) {
+int qlora_quantize_codebook(const float* Wt, const nf4_weight* q, int codebook_id,
+                            qlora_stream_t stream) {
   if (!Wt) return QLORA_ERR_INVALID_ARG;
+  if (codebook_id < 0 || codebook_id >= kCodebooks) return QLORA_ERR_INVALID_ARG;
   int rc = check_weight(q);
   if (rc) return rc;
   if (!aligned16(Wt)) return QLORA_ERR_MISALIGNED;
@@ -671,13 +703,16 @@ int nf4_quantize(const float* Wt, const nf4_weight* q, qlora_stream_t stream) {
   {
     prof::Scope ps(prof::kQuant, reinterpret_cast<cudaStream_t>(stream));
     nf4_quantize_kernel<<<grid, qz::kThreads, qz::smem_bytes(), reinterpret_cast<cudaStream_t>(stream)>>>(
-        Wt, q->codes, q->absmax_q8, q->absmax_s2, nblocks, device_table(), device_buckets());
+        Wt, q->codes, q->absmax_q8, q->absmax_s2, nblocks, device_table(codebook_id),
+        device_buckets(codebook_id));
   }
   return launch_status();
 }
 
-int nf4_dequantize(const nf4_weight* q, uint16_t* Wt_out, qlora_stream_t stream) {
+int qlora_dequantize_codebook(const nf4_weight* q, int codebook_id, uint16_t* Wt_out,
+                              qlora_stream_t stream) {
   if (!Wt_out) return QLORA_ERR_INVALID_ARG;
+  if (codebook_id < 0 || codebook_id >= kCodebooks) return QLORA_ERR_INVALID_ARG;
   int rc = check_weight(q);
   if (rc) return rc;
   if (!aligned16(Wt_out)) return QLORA_ERR_MISALIGNED;
@@ -689,9 +724,25 @@ int nf4_dequantize(const nf4_weight* q, uint16_t* Wt_out, qlora_stream_t stream)
   {
     prof::Scope ps(prof::kDequant, reinterpret_cast<cudaStream_t>(stream));
     nf4_dequantize_kernel<<<std::max(grid, 1), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        q->codes, q->absmax_q8, q->absmax_s2, Wt_out, nitems, device_table());
+        q->codes, q->absmax_q8, q->absmax_s2, Wt_out, nitems, device_table(codebook_id));
   }
   return launch_status();
+}
+
+int nf4_quantize(const float* Wt, const nf4_weight* q, qlora_stream_t stream) {
+  return qlora_quantize_codebook(Wt, q, 0, stream);
+}
+
+int nf4_dequantize(const nf4_weight* q, uint16_t* Wt_out, qlora_stream_t stream) {
+  return qlora_dequantize_codebook(q, 0, Wt_out, stream);
+}
+
+int qlora_codebook(int codebook_id, float* levels, float* midpoints) {
+  if (!levels || codebook_id < 0 || codebook_id >= kCodebooks) return QLORA_ERR_INVALID_ARG;
+  const Codebook& cb = codebook(codebook_id);
+  std::memcpy(levels, cb.level, sizeof(cb.level));
+  if (midpoints) std::memcpy(midpoints, cb.mid, sizeof(cb.mid));
+  return QLORA_OK;
 }
 
 int qlora_linear_fwd(const uint16_t* X, int64_t t, const nf4_weight* W, const uint16_t* L1,

@@ -198,6 +198,27 @@ QLORA_API int qlora_profile_begin(int capacity);
 QLORA_API int qlora_profile_end(double *ms, int64_t *launches, int nkinds);
 QLORA_API const char *qlora_kernel_name(int kind);
 
+/* Other 4-bit codebooks, for the format comparison the pages draw (NF4 against FP4 and INT4:
+ * "QLoRA in LLMs" section 5; "Idea one: NF4", goodomens.studio). Same 64-weight blocks,
+ * packing and double-quantized scales as nf4_quantize / nf4_dequantize; only the 16 levels
+ * (and the code of the zero level, taken by all-zero blocks) differ. codebook_id:
+ *   QLORA_CODEBOOK_NF4 (0)   the NF4 levels (nf4_quantize / nf4_dequantize use these)
+ *   QLORA_CODEBOOK_FP4 (1)   FP4 E2M1: {0, .5, 1, 1.5, 2, 3, 4, 6} with both signs, over 6,
+ *                            -0 and +0 both kept (codes 7 and 8); zero code 7
+ *   QLORA_CODEBOOK_INT4 (2)  absmax INT4: k / 7 for k = -8 .. 7; zero code 8
+ * A weight packed with one codebook must be dequantized with the same one (the packed
+ * format does not record it); only NF4-packed weights may be passed to the linear calls.
+ * qlora_codebook writes that codebook's 16 levels (and 15 midpoints if non-NULL).
+ * Errors: QLORA_ERR_INVALID_ARG for an unknown id, else as nf4_quantize / nf4_dequantize. */
+#define QLORA_CODEBOOK_NF4 0
+#define QLORA_CODEBOOK_FP4 1
+#define QLORA_CODEBOOK_INT4 2
+QLORA_API int qlora_codebook(int codebook_id, float *levels, float *midpoints);
+QLORA_API int qlora_quantize_codebook(const float *Wt, const nf4_weight *q, int codebook_id,
+                                      qlora_stream_t stream);
+QLORA_API int qlora_dequantize_codebook(const nf4_weight *q, int codebook_id, uint16_t *Wt_out,
+                                        qlora_stream_t stream);
+
 /* Adapter merge ("QLoRA in LLMs" section 11, "Saving, Loading, and Merging QLoRA Adapters":
  * dequantize the base into a wider precision, add the LoRA update, optionally quantize the
  * result again): Wt_merged = W'^T + s . (L1 . L2)^T, i.e. W_m = W' + s.L1.L2 in the stored

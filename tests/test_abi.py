@@ -110,3 +110,17 @@ def test_host_validation_rejects_before_launch(lib):
     assert bwd(P, P, 4, ctypes.byref(d), P, P, 16, 1.0, None, P, P, None, P, 1 << 30, None) == B.QLORA_ERR_INVALID_ARG
     assert bwd(P, P, 4, ctypes.byref(d), P, P, 16, 1.0, None, P, P, P + 4, P, 1 << 30, None) == B.QLORA_ERR_MISALIGNED
     assert bwd(P, P, 4, ctypes.byref(d), P, P, 16, 1.0, None, P, P, P, P, 8, None) == B.QLORA_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("cb", [0, 1, 2])
+def test_codebooks_match_oracle_bit_exactly(lib, cb):
+    lv, md = B.codebook(cb)
+    want = O.codebook_levels(cb)
+    assert np.array_equal(np.array(lv, np.float32).view(np.uint32), want.view(np.uint32))
+    assert np.array_equal(np.array(md, np.float32).view(np.uint32), O.nf4_midpoints(want).view(np.uint32))
+
+
+def test_unknown_codebook_is_rejected(lib):
+    lv = (ctypes.c_float * 16)()
+    assert lib.qlora_codebook(3, ctypes.cast(lv, ctypes.c_void_p), None) == B.QLORA_ERR_INVALID_ARG
+    assert lib.qlora_codebook(-1, ctypes.cast(lv, ctypes.c_void_p), None) == B.QLORA_ERR_INVALID_ARG

@@ -110,3 +110,29 @@ def test_sampled_rows_of_the_largest_decode_weight():
     ref = oracle_packed_rows(Wt.numpy(), rows)
     got = deq[rows].float().cpu().numpy()
     assert np.array_equal(got.view(np.uint32), ref.astype(np.float32).view(np.uint32))
+
+
+def _check_codebook(Wt: torch.Tensor, cb: int):
+    p = B.nf4_quantize(Wt.cuda(), codebook_id=cb)
+    deq = B.nf4_dequantize(p, codebook_id=cb)
+    assert B.last_status() == 0
+    ref = O.quantize_with(Wt.numpy(), cb)
+    assert np.array_equal(p.codes.cpu().numpy(), ref.codes), "packed codes differ"
+    assert np.array_equal(p.absmax_q8.cpu().numpy(), ref.absmax_q8), "8-bit scales differ"
+    assert np.array_equal(p.absmax_s2.cpu().numpy().view(np.uint32),
+                          ref.absmax_s2.view(np.uint32)), "second-level scales differ"
+    got = deq.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got.reshape(-1), O.dequantize_bits_with(ref, cb).reshape(-1)), \
+        "dequantized bf16 differs"
+
+
+@pytest.mark.parametrize("cb", [B.CODEBOOK_FP4, B.CODEBOOK_INT4])
+def test_other_codebooks_bit_exact(cb):
+    """FP4 and INT4 packing, bit for bit: a LLaMA-7B q_proj with 1% outliers, a ragged shape,
+    and rows with all-zero blocks (the codebook's own zero code)."""
+    _check_codebook(inputs.weight_f32(4096, 4096, 200, outliers=True), cb)
+    g = torch.Generator().manual_seed(cb)
+    W = torch.randn(257, 192, generator=g) * 0.02
+    W[3] = 0.0
+    W[10, :64] = 0.0
+    _check_codebook(W, cb)
