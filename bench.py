@@ -375,6 +375,37 @@ def stack65b_leg(dev, peaks, steps: int = 2, warmup: int = 1):
     return res
 
 
+def codebook_leg(dev):
+    """The pages' format comparison on the LLaMA-7B-shaped layer's weights: relative
+    reconstruction error (sum of squared errors / sum of squares) of NF4, FP4 and INT4 packing
+    (same blocks and double-quantized scales), on N(0, 0.02) weights with the 1% outliers at
+    8 sigma of the quantization workload and without them, and the quantizer's time for each."""
+    from bit_quantized_lora_03_b200 import binding as B
+    from bit_quantized_lora_03_b200 import inputs
+    res = {}
+    for tag, outl in (("with_outliers", True), ("gaussian", False)):
+        W = [w.to(dev) for _, w in inputs.llama7b_quant_weights(with_outliers=outl)]
+        res[tag] = {}
+        for name, cb in (("nf4", B.CODEBOOK_NF4), ("fp4", B.CODEBOOK_FP4), ("int4", B.CODEBOOK_INT4)):
+            packs = [B.PackedNF4(w.shape[0], w.shape[1], dev) for w in W]
+
+            def quant():
+                for w, p in zip(W, packs):
+                    B.nf4_quantize(w, out=p, codebook_id=cb)
+            ms = queued_ms(quant, 3, 1) / 3
+            se, ss = 0.0, 0.0
+            for w, p in zip(W, packs):
+                d = B.nf4_dequantize(p, codebook_id=cb).float()
+                se += float((d - w).pow(2).sum())
+                ss += float(w.pow(2).sum())
+            res[tag][name] = {"rel_mse": round(se / ss, 6), "quantize_ms": round(ms, 4)}
+            del packs
+        del W
+        torch.cuda.empty_cache()
+    res["device_status"] = B.last_status()
+    return res
+
+
 def merge_leg(dev, peaks, r: int = 64, s: float = 0.25):
     """Adapter merge over the 7 linears of the LLaMA-7B-shaped layer: GB/s of the merge
     (write 4 B + read 0.516 B per weight) and of the re-quantization, and the output drift of
@@ -630,6 +661,7 @@ def main():
         legs["codec_llama7b_layer"] = codec_leg(dev, peaks)
         legs["stack65b"] = stack65b_leg(dev, peaks)
         legs["merge_llama7b_layer"] = merge_leg(dev, peaks)
+        legs["codebooks_llama7b_layer"] = codebook_leg(dev)
         tps, sec, _ = oracle_sample(args.cpu_sample_tokens)
         cpu = {"value": round(tps, 3), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                "sample": (f"fwd+bwd of {args.cpu_sample_tokens} of the 4096 tokens, one linear per "
