@@ -458,6 +458,26 @@ def merge_error_bound(Wdq, L1, L2, s):
     return 2.0 * (r + 2) * 2.0 ** -24 * mag
 
 
+# ----------------------------------------------------------------------------------------
+# Adapter update with a paged optimizer ("QLoRA in LLMs" §4 "Update the adapters" and §7 "Paged
+# Optimizers Manage Temporary Memory Spikes"; "Idea three: paged optimizers", goodomens.studio).
+# The pages name the optimizer state ("running statistics") but not the rule; the reading is
+# AdamW (decoupled weight decay, bias-corrected moments), the optimizer QLoRA pages.
+# ----------------------------------------------------------------------------------------
+
+def adamw_step(p, g, m, v, step, lr, beta1, beta2, eps, weight_decay):
+    """One AdamW update in fp64; returns (p, m, v) after step `step` (1-based):
+    p <- p (1 - lr wd);  m <- b1 m + (1 - b1) g;  v <- b2 v + (1 - b2) g^2;
+    p <- p - lr * (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps)."""
+    p, g, m, v = _f64(p), _f64(g), _f64(m), _f64(v)
+    p = p * (1.0 - lr * weight_decay)
+    m = beta1 * m + (1.0 - beta1) * g
+    v = beta2 * v + (1.0 - beta2) * g * g
+    mhat = m / (1.0 - beta1 ** step)
+    vhat = v / (1.0 - beta2 ** step)
+    return p - lr * mhat / (np.sqrt(vhat) + eps), m, v
+
+
 def max_err_vs_rms(got, ref) -> tuple[float, float]:
     """(max |got - ref|, RMS(ref)) in fp64: the tolerance test is max <= 2e-2 * RMS."""
     got, ref = _f64(got), _f64(ref)
