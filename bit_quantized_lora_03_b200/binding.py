@@ -48,6 +48,9 @@ SIGNATURES = {
     "qlora_selftest_wait_timeout": (ctypes.c_int, [_I64, _PTR]),
     "qlora_merge_adapters": (ctypes.c_int, [_PTR, _PTR, _PTR, _I64, ctypes.c_float, _PTR, _PTR]),
     "qlora_codebook": (ctypes.c_int, [ctypes.c_int, _PTR, _PTR]),
+    "qlora_adamw_step": (ctypes.c_int, [_PTR, _PTR, _PTR, _PTR, _PTR, _I64, ctypes.c_float,
+                                        ctypes.c_float, ctypes.c_float, ctypes.c_float,
+                                        ctypes.c_float, _I64, _PTR]),
     "qlora_quantize_codebook": (ctypes.c_int, [_PTR, _PTR, ctypes.c_int, _PTR]),
     "qlora_dequantize_codebook": (ctypes.c_int, [_PTR, ctypes.c_int, _PTR, _PTR]),
     "qlora_profile_begin": (ctypes.c_int, [ctypes.c_int]),
@@ -307,6 +310,28 @@ def merge_adapters(p: PackedNF4, L1: torch.Tensor, L2: torch.Tensor, s: float,
                                       float(s), out.data_ptr(), _stream(stream)),
            "qlora_merge_adapters")
     return out
+
+
+def adamw_step_ptr(p: int, p16: int, g: int, m: int, v: int, n: int, lr: float, beta1: float,
+                   beta2: float, eps: float, weight_decay: float, step: int, stream=None) -> None:
+    """qlora_adamw_step on raw device (or unified-memory) pointers."""
+    _check(lib().qlora_adamw_step(p, p16, g, m, v, int(n), float(lr), float(beta1), float(beta2),
+                                  float(eps), float(weight_decay), int(step), _stream(stream)),
+           "qlora_adamw_step")
+
+
+def adamw_step(p: torch.Tensor, g: torch.Tensor, m: torch.Tensor, v: torch.Tensor, step: int,
+               lr: float = 1e-4, beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8,
+               weight_decay: float = 0.0, p16: torch.Tensor | None = None, stream=None) -> None:
+    """One fused AdamW step on fp32 CUDA tensors of equal shape (in place); p16, if given, gets
+    the bf16 copy of the updated parameters."""
+    for t, name in ((p, "p"), (g, "g"), (m, "m"), (v, "v")):
+        _require(t, torch.float32, p.shape, name)
+    if p16 is not None:
+        _require(p16, torch.bfloat16, p.shape, "p16")
+    adamw_step_ptr(p.data_ptr(), p16.data_ptr() if p16 is not None else 0, g.data_ptr(),
+                   m.data_ptr(), v.data_ptr(), p.numel(), lr, beta1, beta2, eps, weight_decay,
+                   step, stream)
 
 
 def selftest_wait_timeout(limit_ns: int, stream=None) -> None:

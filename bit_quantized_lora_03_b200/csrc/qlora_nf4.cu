@@ -18,6 +18,7 @@
 #include "nf4_codec.cuh"
 #include "nf4_gemm.cuh"
 #include "tc_gemm.cuh"
+#include "adamw.cuh"
 #include "nf4_gemv.cuh"
 
 using namespace qlora;
@@ -561,6 +562,57 @@ int qlora_merge_adapters(const nf4_weight* W, const uint16_t* L1, const uint16_t
     return QLORA_ERR_CUDA;
   return launch_tc_gemm<true, false>(mA, mB, o, h, pl, s, kOutMergeNF4, Wt_merged, h, nullptr,
                                      nullptr, kPdlNone, st, W);
+}
+
+// Bring a buffer in unified (managed) memory to this device before a kernel touches it, as a
+// paged optimizer's state returns when the optimizer needs it; plain device memory is left as
+// it is. Pure hints: a failed query or prefetch changes nothing but speed.
+void prefetch_if_managed(const void* ptr, size_t bytes, int dev, cudaStream_t st) {
+  cudaPointerAttributes at{};
+  if (cudaPointerGetAttributes(&at, ptr) != cudaSuccess) {
+    cudaGetLastError();
+    return;
+  }
+  if (at.type == cudaMemoryTypeManaged && cudaMemPrefetchAsync(ptr, bytes, dev, st) != cudaSuccess)
+    cudaGetLastError();
+}
+
+int qlora_adamw_step(float* param, uint16_t* param_bf16, const float* grad, float* m, float* v,
+                     int64_t n, float lr, float beta1, float beta2, float eps, float weight_decay,
+                     int64_t step, qlora_stream_t stream) {
+  if (!param || !grad || !m || !v || n <= 0 || n % 4 != 0 || step < 1) return QLORA_ERR_INVALID_ARG;
+  if (!std::isfinite(lr) || !std::isfinite(eps) || !std::isfinite(weight_decay) || eps <= 0.f ||
+      !(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f))
+    return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(param) || !aligned16(grad) || !aligned16(m) || !aligned16(v) ||
+      (param_bf16 && (reinterpret_cast<uintptr_t>(param_bf16) & 7u)))
+    return QLORA_ERR_MISALIGNED;
+  int dev, rc;
+  if ((rc = current_device(&dev))) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t bytes = static_cast<size_t>(n) * 4;
+  prefetch_if_managed(m, bytes, dev, st);
+  prefetch_if_managed(v, bytes, dev, st);
+  prefetch_if_managed(param, bytes, dev, st);
+  prefetch_if_managed(grad, bytes, dev, st);
+  AdamwArgs a{};
+  a.p = param;
+  a.p16 = param_bf16;
+  a.g = grad;
+  a.m = m;
+  a.v = v;
+  a.n4 = n / 4;
+  a.lr = lr;
+  a.beta1 = beta1;
+  a.beta2 = beta2;
+  a.eps = eps;
+  a.wd = weight_decay;
+  a.step_size = static_cast<float>(lr / (1.0 - std::pow(static_cast<double>(beta1), static_cast<double>(step))));
+  a.inv_sqrt_bc2 = static_cast<float>(1.0 / std::sqrt(1.0 - std::pow(static_cast<double>(beta2), static_cast<double>(step))));
+  const int64_t want = (a.n4 + 255) / 256;
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(sm_count(dev)) * 8)));
+  adamw_kernel<<<grid, 256, 0, st>>>(a);
+  return launch_status();
 }
 
 // One thread waits on an mbarrier that no arrival will ever complete; the bounded wait gives

@@ -235,6 +235,25 @@ QLORA_API int qlora_dequantize_codebook(const nf4_weight *q, int codebook_id, ui
 QLORA_API int qlora_merge_adapters(const nf4_weight *W, const uint16_t *L1, const uint16_t *L2,
                                    int64_t r, float s, float *Wt_merged, qlora_stream_t stream);
 
+/* Adapter update with a paged optimizer ("QLoRA in LLMs" sections 4 and 7; "Idea three: paged
+ * optimizers", goodomens.studio): one fused AdamW step over n fp32 parameters (an adapter,
+ * e.g. L1 with n = h * r, using its dL1 as grad), with decoupled weight decay and bias-corrected
+ * moments at 1-based step t:
+ *   p <- p (1 - lr wd);  m <- b1 m + (1 - b1) g;  v <- b2 v + (1 - b2) g^2;
+ *   p <- p - (lr / (1 - b1^t)) m / (sqrt(v) / sqrt(1 - b2^t) + eps)
+ * and, if param_bf16 is non-NULL, its bf16 copy (round to nearest even) for the next forward.
+ * The pages name the optimizer state but not the rule; AdamW is the reading. Any buffer may be
+ * unified (cudaMallocManaged) memory, as the pages' paged optimizer keeps its state: such a
+ * buffer is prefetched to the current device on `stream` before the update, and the driver may
+ * move it back to host memory afterwards under memory pressure. param, grad, m, v: 16-byte
+ * aligned, caller-owned, n % 4 == 0; param, m, v, param_bf16 are updated in place.
+ * Errors: QLORA_ERR_INVALID_ARG (null, n, step < 1, eps <= 0, betas outside [0, 1)),
+ * QLORA_ERR_MISALIGNED, QLORA_ERR_CUDA; nothing is launched on an error. */
+QLORA_API int qlora_adamw_step(float *param, uint16_t *param_bf16, const float *grad, float *m,
+                               float *v, int64_t n, float lr, float beta1, float beta2,
+                               float eps, float weight_decay, int64_t step,
+                               qlora_stream_t stream);
+
 /* Launch shape of the decode GEMV (t <= 16), a scheduling knob with no counterpart in the
  * method. By default the GEMV runs one CTA of 16 warps per SM and splits its units (32 rows x
  * 128 inputs) evenly over all their warps. qlora_set_gemv_max_ctas(n) caps that CTA count at

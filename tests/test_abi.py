@@ -124,3 +124,19 @@ def test_unknown_codebook_is_rejected(lib):
     lv = (ctypes.c_float * 16)()
     assert lib.qlora_codebook(3, ctypes.cast(lv, ctypes.c_void_p), None) == B.QLORA_ERR_INVALID_ARG
     assert lib.qlora_codebook(-1, ctypes.cast(lv, ctypes.c_void_p), None) == B.QLORA_ERR_INVALID_ARG
+
+
+def test_adamw_argument_checks(lib):
+    f = lib.qlora_adamw_step
+    p = ctypes.c_void_p(16)   # never dereferenced: the checks run before anything else
+    ok = dict(lr=1e-3, b1=0.9, b2=0.999, eps=1e-8, wd=0.0)
+
+    def call(n=64, step=1, lr=ok["lr"], b1=ok["b1"], b2=ok["b2"], eps=ok["eps"], ptr=p):
+        return f(ptr, None, ptr, ptr, ptr, n, lr, b1, b2, eps, ok["wd"], step, None)
+    assert call(n=6) == B.QLORA_ERR_INVALID_ARG          # n % 4 != 0
+    assert call(step=0) == B.QLORA_ERR_INVALID_ARG
+    assert call(eps=0.0) == B.QLORA_ERR_INVALID_ARG
+    assert call(b1=1.0) == B.QLORA_ERR_INVALID_ARG
+    assert call(lr=float("nan")) == B.QLORA_ERR_INVALID_ARG
+    assert call(ptr=None) == B.QLORA_ERR_INVALID_ARG
+    assert call(ptr=ctypes.c_void_p(20)) == B.QLORA_ERR_MISALIGNED
