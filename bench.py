@@ -406,6 +406,72 @@ def codebook_leg(dev):
     return res
 
 
+def adamw_leg(dev, peaks, r: int = 64):
+    """The adapters' update for the 7-linear layer (L1 and L2 of every linear: sum r (h + o) =
+    4.997 M parameters): device time of one fused AdamW step over all 14 adapters with the
+    state in device memory, with it in unified memory resident on the GPU, and with it in
+    unified memory paged out to the host first (the paged optimizer's spike path)."""
+    import ctypes
+    from bit_quantized_lora_03_b200 import binding as B
+    from bit_quantized_lora_03_b200 import inputs
+    from cuda.bindings import runtime as rt
+    sizes = [n for _, h, o in inputs.LLAMA7B_LINEARS for n in (h * r, r * o)]
+    total = sum(sizes)
+    p = [torch.randn(n, device=dev) * 0.01 for n in sizes]
+    g = [torch.randn(n, device=dev) * 0.01 for n in sizes]
+    p16 = [torch.empty(n, dtype=torch.bfloat16, device=dev) for n in sizes]
+    md = [torch.zeros(n, device=dev) for n in sizes]
+    vd = [torch.zeros(n, device=dev) for n in sizes]
+    mu, vu = [], []
+    for n in sizes:
+        for lst in (mu, vu):
+            err, ptr = rt.cudaMallocManaged(4 * n, rt.cudaMemAttachGlobal)
+            assert err == rt.cudaError_t.cudaSuccess
+            ctypes.memset(int(ptr), 0, 4 * n)
+            lst.append(int(ptr))
+    step = [0]
+
+    def run(ms, vs, flags=0):
+        step[0] += 1
+        for i, n in enumerate(sizes):
+            B.adamw_step_ptr(p[i].data_ptr(), p16[i].data_ptr(), g[i].data_ptr(),
+                             ms[i] if isinstance(ms[i], int) else ms[i].data_ptr(),
+                             vs[i] if isinstance(vs[i], int) else vs[i].data_ptr(),
+                             n, 1e-4, 0.9, 0.999, 1e-8, 0.0, step[0], flags)
+
+    def paged_in(flags):
+        """One step after the state was moved to host memory."""
+        torch.cuda.synchronize()
+        for ptr, n in zip(mu + vu, sizes + sizes):
+            rt.cudaMemPrefetchAsync(ptr, 4 * n, rt.cudaCpuDeviceId, 0)
+        torch.cuda.synchronize()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record()
+        run(mu, vu, flags)
+        end.record()
+        torch.cuda.synchronize()
+        return start.elapsed_time(end)
+
+    dev_ms = queued_ms(lambda: run(md, vd), 5, 2) / 5
+    uni_ms = queued_ms(lambda: run(mu, vu), 5, 2) / 5
+    uni_pf_ms = queued_ms(lambda: run(mu, vu, B.ADAMW_PREFETCH), 5, 2) / 5
+    paged_fault_ms = paged_in(0)
+    paged_pf_ms = paged_in(B.ADAMW_PREFETCH)
+    status = B.last_status()
+    for ptr in mu + vu:
+        rt.cudaFree(ptr)
+    nbytes = 30 * total   # read p, g, m, v; write p, m, v (fp32) and the bf16 copy
+    return {"params": total, "bytes_per_step": nbytes,
+            "device_state_ms": round(dev_ms, 4),
+            "device_state_gbs": round(nbytes / (dev_ms * 1e-3) / 1e9, 1),
+            "device_state_frac_hbm": round(nbytes / (dev_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
+            "unified_state_resident_ms": round(uni_ms, 4),
+            "unified_state_resident_prefetch_ms": round(uni_pf_ms, 4),
+            "unified_state_paged_out_first_touch_ms": round(paged_fault_ms, 4),
+            "unified_state_paged_out_prefetch_ms": round(paged_pf_ms, 4),
+            "device_status": status}
+
+
 def merge_leg(dev, peaks, r: int = 64, s: float = 0.25):
     """Adapter merge over the 7 linears of the LLaMA-7B-shaped layer: GB/s of the merge
     (write 4 B + read 0.516 B per weight) and of the re-quantization, and the output drift of
@@ -662,6 +728,7 @@ def main():
         legs["stack65b"] = stack65b_leg(dev, peaks)
         legs["merge_llama7b_layer"] = merge_leg(dev, peaks)
         legs["codebooks_llama7b_layer"] = codebook_leg(dev)
+        legs["adamw_llama7b_adapters"] = adamw_leg(dev, peaks)
         tps, sec, _ = oracle_sample(args.cpu_sample_tokens)
         cpu = {"value": round(tps, 3), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                "sample": (f"fwd+bwd of {args.cpu_sample_tokens} of the 4096 tokens, one linear per "

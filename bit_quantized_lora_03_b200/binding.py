@@ -50,7 +50,7 @@ SIGNATURES = {
     "qlora_codebook": (ctypes.c_int, [ctypes.c_int, _PTR, _PTR]),
     "qlora_adamw_step": (ctypes.c_int, [_PTR, _PTR, _PTR, _PTR, _PTR, _I64, ctypes.c_float,
                                         ctypes.c_float, ctypes.c_float, ctypes.c_float,
-                                        ctypes.c_float, _I64, _PTR]),
+                                        ctypes.c_float, _I64, ctypes.c_uint, _PTR]),
     "qlora_quantize_codebook": (ctypes.c_int, [_PTR, _PTR, ctypes.c_int, _PTR]),
     "qlora_dequantize_codebook": (ctypes.c_int, [_PTR, ctypes.c_int, _PTR, _PTR]),
     "qlora_profile_begin": (ctypes.c_int, [ctypes.c_int]),
@@ -312,11 +312,16 @@ def merge_adapters(p: PackedNF4, L1: torch.Tensor, L2: torch.Tensor, s: float,
     return out
 
 
+ADAMW_PREFETCH = 1
+
+
 def adamw_step_ptr(p: int, p16: int, g: int, m: int, v: int, n: int, lr: float, beta1: float,
-                   beta2: float, eps: float, weight_decay: float, step: int, stream=None) -> None:
+                   beta2: float, eps: float, weight_decay: float, step: int, flags: int = 0,
+                   stream=None) -> None:
     """qlora_adamw_step on raw device (or unified-memory) pointers."""
     _check(lib().qlora_adamw_step(p, p16, g, m, v, int(n), float(lr), float(beta1), float(beta2),
-                                  float(eps), float(weight_decay), int(step), _stream(stream)),
+                                  float(eps), float(weight_decay), int(step), int(flags),
+                                  _stream(stream)),
            "qlora_adamw_step")
 
 
@@ -331,7 +336,7 @@ def adamw_step(p: torch.Tensor, g: torch.Tensor, m: torch.Tensor, v: torch.Tenso
         _require(p16, torch.bfloat16, p.shape, "p16")
     adamw_step_ptr(p.data_ptr(), p16.data_ptr() if p16 is not None else 0, g.data_ptr(),
                    m.data_ptr(), v.data_ptr(), p.numel(), lr, beta1, beta2, eps, weight_decay,
-                   step, stream)
+                   step, 0, stream)
 
 
 def selftest_wait_timeout(limit_ns: int, stream=None) -> None:

@@ -579,7 +579,7 @@ void prefetch_if_managed(const void* ptr, size_t bytes, int dev, cudaStream_t st
 
 int qlora_adamw_step(float* param, uint16_t* param_bf16, const float* grad, float* m, float* v,
                      int64_t n, float lr, float beta1, float beta2, float eps, float weight_decay,
-                     int64_t step, qlora_stream_t stream) {
+                     int64_t step, unsigned flags, qlora_stream_t stream) {
   if (!param || !grad || !m || !v || n <= 0 || n % 4 != 0 || step < 1) return QLORA_ERR_INVALID_ARG;
   if (!std::isfinite(lr) || !std::isfinite(eps) || !std::isfinite(weight_decay) || eps <= 0.f ||
       !(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f))
@@ -590,11 +590,14 @@ int qlora_adamw_step(float* param, uint16_t* param_bf16, const float* grad, floa
   int dev, rc;
   if ((rc = current_device(&dev))) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const size_t bytes = static_cast<size_t>(n) * 4;
-  prefetch_if_managed(m, bytes, dev, st);
-  prefetch_if_managed(v, bytes, dev, st);
-  prefetch_if_managed(param, bytes, dev, st);
-  prefetch_if_managed(grad, bytes, dev, st);
+  if (flags & ~static_cast<unsigned>(QLORA_ADAMW_PREFETCH)) return QLORA_ERR_INVALID_ARG;
+  if (flags & QLORA_ADAMW_PREFETCH) {
+    const size_t bytes = static_cast<size_t>(n) * 4;
+    prefetch_if_managed(m, bytes, dev, st);
+    prefetch_if_managed(v, bytes, dev, st);
+    prefetch_if_managed(param, bytes, dev, st);
+    prefetch_if_managed(grad, bytes, dev, st);
+  }
   AdamwArgs a{};
   a.p = param;
   a.p16 = param_bf16;

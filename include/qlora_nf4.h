@@ -243,15 +243,19 @@ QLORA_API int qlora_merge_adapters(const nf4_weight *W, const uint16_t *L1, cons
  *   p <- p - (lr / (1 - b1^t)) m / (sqrt(v) / sqrt(1 - b2^t) + eps)
  * and, if param_bf16 is non-NULL, its bf16 copy (round to nearest even) for the next forward.
  * The pages name the optimizer state but not the rule; AdamW is the reading. Any buffer may be
- * unified (cudaMallocManaged) memory, as the pages' paged optimizer keeps its state: such a
- * buffer is prefetched to the current device on `stream` before the update, and the driver may
- * move it back to host memory afterwards under memory pressure. param, grad, m, v: 16-byte
- * aligned, caller-owned, n % 4 == 0; param, m, v, param_bf16 are updated in place.
- * Errors: QLORA_ERR_INVALID_ARG (null, n, step < 1, eps <= 0, betas outside [0, 1)),
- * QLORA_ERR_MISALIGNED, QLORA_ERR_CUDA; nothing is launched on an error. */
+ * unified (cudaMallocManaged) memory, as the pages' paged optimizer keeps its state: the kernel
+ * then reads it wherever the driver has placed it (pages on the host migrate on first touch),
+ * and with flags = QLORA_ADAMW_PREFETCH each unified buffer is first prefetched to the current
+ * device on `stream` (bulk migration; on pages already resident the prefetch still costs
+ * driver time). The driver may move the state back to host memory under memory pressure.
+ * param, grad, m, v: 16-byte aligned, caller-owned, n % 4 == 0; param, m, v, param_bf16 are
+ * updated in place. Hyper-parameters are used as the fp32 values given.
+ * Errors: QLORA_ERR_INVALID_ARG (null, n, step < 1, eps <= 0, betas outside [0, 1), unknown
+ * flags), QLORA_ERR_MISALIGNED, QLORA_ERR_CUDA; nothing is launched on an error. */
+#define QLORA_ADAMW_PREFETCH 1u
 QLORA_API int qlora_adamw_step(float *param, uint16_t *param_bf16, const float *grad, float *m,
                                float *v, int64_t n, float lr, float beta1, float beta2,
-                               float eps, float weight_decay, int64_t step,
+                               float eps, float weight_decay, int64_t step, unsigned flags,
                                qlora_stream_t stream);
 
 /* Launch shape of the decode GEMV (t <= 16), a scheduling knob with no counterpart in the

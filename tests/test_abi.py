@@ -132,7 +132,7 @@ def test_adamw_argument_checks(lib):
     ok = dict(lr=1e-3, b1=0.9, b2=0.999, eps=1e-8, wd=0.0)
 
     def call(n=64, step=1, lr=ok["lr"], b1=ok["b1"], b2=ok["b2"], eps=ok["eps"], ptr=p):
-        return f(ptr, None, ptr, ptr, ptr, n, lr, b1, b2, eps, ok["wd"], step, None)
+        return f(ptr, None, ptr, ptr, ptr, n, lr, b1, b2, eps, ok["wd"], step, 0, None)
     assert call(n=6) == B.QLORA_ERR_INVALID_ARG          # n % 4 != 0
     assert call(step=0) == B.QLORA_ERR_INVALID_ARG
     assert call(eps=0.0) == B.QLORA_ERR_INVALID_ARG

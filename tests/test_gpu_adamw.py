@@ -69,11 +69,13 @@ def test_adamw_with_state_in_unified_memory():
         m_b, v_b = torch.zeros(n, device="cuda"), torch.zeros(n, device="cuda")
         for t, g in enumerate(_grads(n, 3, 10), start=1):
             gd = g.cuda()
-            if t == 2:   # page the state out to host memory; the step brings it back
+            if t >= 2:   # page the state out to host memory; the step brings it back
                 for ptr in (m_ptr, v_ptr):
                     assert rt.cudaMemPrefetchAsync(ptr, 4 * n, rt.cudaCpuDeviceId, 0)[0] == rt.cudaError_t.cudaSuccess
+            # step 2 prefetches the paged-out state back; step 3 lets it migrate on first touch
             B.adamw_step_ptr(p_a.data_ptr(), 0, gd.data_ptr(), m_ptr, v_ptr, n, HP["lr"],
-                             HP["beta1"], HP["beta2"], HP["eps"], HP["weight_decay"], t)
+                             HP["beta1"], HP["beta2"], HP["eps"], HP["weight_decay"], t,
+                             flags=B.ADAMW_PREFETCH if t == 2 else 0)
             B.adamw_step(p_b, gd, m_b, v_b, t, **HP)
         assert B.last_status() == 0
         torch.cuda.synchronize()
