@@ -593,6 +593,24 @@ def run_reference(args, rank):
     return 0
 
 
+def decode_case(B, dev, t, wi):
+    """A short decode run for one capture: the third GEMV launch is the steady state."""
+    from bit_quantized_lora_03_b200 import inputs
+    name, Wt = inputs.decode_gemv_weights()[wi]
+    o, h = Wt.shape
+    p = B.nf4_quantize(Wt.to(dev))
+    del Wt
+    L1, L2 = (a.to(dev) for a in inputs.decode_gemv_adapters(h, o, 16))
+    X = inputs.decode_gemv_activations(h, t).to(dev)
+    for _ in range(3):
+        B.qlora_linear_fwd(X, p, L1, L2, 2.0, want_sT=False)
+    torch.cuda.synchronize()
+    status = B.last_status()
+    print(json.dumps({"case": f"decode {name} o={o} h={h} t={t}", "device_status": status}),
+          flush=True)
+    return 0 if status == 0 else 1
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -606,6 +624,9 @@ def main():
                     help="streams the 7 independent linears of a step are spread over")
     ap.add_argument("--single-linear", type=int, default=None, metavar="I",
                     help="profiling case: only linear I of the layer, fwd+bwd, no extras")
+    ap.add_argument("--decode-case", type=int, nargs=2, default=None, metavar=("T", "I"),
+                    help="profiling case: quantize decode weight I, then three forward calls "
+                         "at T tokens")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -627,6 +648,8 @@ def main():
     props = torch.cuda.get_device_properties(dev)
     l2_bytes = getattr(props, "L2_cache_size", 126 * 2**20)
 
+    if args.decode_case is not None:
+        return decode_case(B, dev, *args.decode_case)
     t, r, s = args.tokens, 64, 0.25
     if args.single_linear is not None:
         L = Layer(args.single_linear, dev, t, r, s)
