@@ -478,6 +478,98 @@ def adamw_step(p, g, m, v, step, lr, beta1, beta2, eps, weight_decay):
     return p - lr * mhat / (np.sqrt(vhat) + eps), m, v
 
 
+# ----------------------------------------------------------------------------------------
+# LoRA dropout on the adapter input ("QLoRA in LLMs" §12 "Minimal QLoRA Setup with Hugging
+# Face": the example configuration sets a LoRA dropout of 0.05; "What it added up to",
+# goodomens.studio, lists dropout among the adapter knobs). The pages do not say where the
+# dropout acts; the reading is the adapter branch's input, inverted scaling:
+#   Y = X.W' + s.(D(X).L1).L2,   D(X) = X (.) M / (1 - p),
+# M a keep mask with P(keep) = 1 - p, drawn by a counter-based generator so that the forward
+# and backward passes (and the oracle) draw the same mask without storing it.
+# ----------------------------------------------------------------------------------------
+
+# Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3",
+# SC'11): a 4 x 32-bit counter is mixed under a 2 x 32-bit key by ten rounds; each round
+# multiplies two counter words by fixed odd constants, keeps both halves of the 64-bit
+# products and XORs the high halves into the other two words together with the key; the key
+# is advanced by two Weyl constants between rounds.
+PHILOX_M0, PHILOX_M1 = 0xD2511F53, 0xCD9E8D57
+PHILOX_W0, PHILOX_W1 = 0x9E3779B9, 0xBB67AE85
+_MASK32 = np.uint64(0xFFFFFFFF)
+
+
+def philox4x32_10(ctr, key):
+    """Philox4x32 with 10 rounds. ctr: (n, 4) uint32 counters; key: (2,) or (n, 2) uint32.
+    Returns (n, 4) uint32."""
+    c = [np.asarray(ctr, dtype=np.uint64)[:, i].copy() for i in range(4)]
+    k = np.broadcast_to(np.asarray(key, dtype=np.uint64), (c[0].shape[0], 2))
+    k0, k1 = k[:, 0].copy(), k[:, 1].copy()
+    for rnd in range(10):
+        if rnd > 0:
+            k0 = (k0 + np.uint64(PHILOX_W0)) & _MASK32
+            k1 = (k1 + np.uint64(PHILOX_W1)) & _MASK32
+        p0 = np.uint64(PHILOX_M0) * c[0]          # exact: both factors < 2^32
+        p1 = np.uint64(PHILOX_M1) * c[2]
+        hi0, lo0 = p0 >> np.uint64(32), p0 & _MASK32
+        hi1, lo1 = p1 >> np.uint64(32), p1 & _MASK32
+        c = [hi1 ^ c[1] ^ k0, lo1, hi0 ^ c[3] ^ k1, lo0]
+    return np.stack(c, axis=1).astype(np.uint32)
+
+
+def dropout_threshold(p) -> int:
+    """Drop an element when its 32-bit draw is below floor(p * 2^32) (p as fp32, 0 <= p < 1),
+    so that P(drop) = threshold / 2^32, within 2^-32 of p."""
+    p = float(np.float32(p))
+    if not (0.0 <= p < 1.0):
+        raise ValueError("dropout probability must lie in [0, 1)")
+    return int(np.floor(p * 4294967296.0))
+
+
+def dropout_keep_mask(t: int, h: int, p, seed: int) -> np.ndarray:
+    """Keep mask M (t x h bool) of the adapter input. Element e = i*h + j (row-major) takes
+    word e mod 4 of Philox4x32-10 at counter (lo32(e div 4), hi32(e div 4), 0, 0) under key
+    (lo32(seed), hi32(seed)); it is kept when that word is >= dropout_threshold(p)."""
+    n = t * h
+    thr = dropout_threshold(p)
+    e = np.arange(n, dtype=np.uint64)
+    groups = np.arange((n + 3) // 4, dtype=np.uint64)
+    ctr = np.zeros((groups.size, 4), dtype=np.uint64)
+    ctr[:, 0] = groups & _MASK32
+    ctr[:, 1] = groups >> np.uint64(32)
+    seed = int(seed) & 0xFFFFFFFFFFFFFFFF
+    words = philox4x32_10(ctr, (seed & 0xFFFFFFFF, seed >> 32))
+    draw = words[(e >> np.uint64(2)).astype(np.int64), (e & np.uint64(3)).astype(np.int64)]
+    return (draw.astype(np.int64) >= thr).reshape(t, h)
+
+
+def dropout_scale(p) -> float:
+    """1 / (1 - p) in fp64 for the fp32 value of p."""
+    return 1.0 / (1.0 - float(np.float32(p)))
+
+
+def qlora_linear_fwd_dropout(X, Wdq, L1, L2, s, keep, p):
+    """Y = X.W' + s.((X (.) M / (1 - p)).L1).L2 in fp64, M = keep.
+    Returns (Y t x o, sT = s.(X (.) M / (1 - p)).L1 t x r)."""
+    X, Wt, L1, L2 = _f64(X), _f64(Wdq), _f64(L1), _f64(L2)
+    Xd = X * np.asarray(keep, dtype=np.float64) * dropout_scale(p)
+    T = Xd @ L1
+    return X @ Wt.T + s * (T @ L2), s * T
+
+
+def qlora_linear_bwd_dropout(dY, X, Wdq, L1, L2, s, keep, p):
+    """Gradients of <dY, Y> for the dropout forward above, in fp64:
+    dX = dY.W'^T + M (.) (s / (1 - p)).(dY.L2^T).L1^T;  dL1 = s.D(X)^T.(dY.L2^T);
+    dL2 = s.(D(X).L1)^T.dY. Returns (dX, dL1, dL2)."""
+    dY, X, Wt, L1, L2 = _f64(dY), _f64(X), _f64(Wdq), _f64(L1), _f64(L2)
+    M = np.asarray(keep, dtype=np.float64) * dropout_scale(p)
+    Xd = X * M
+    U = dY @ L2.T
+    dX = dY @ Wt + M * (s * (U @ L1.T))
+    dL1 = s * (Xd.T @ U)
+    dL2 = s * ((Xd @ L1).T @ dY)
+    return dX, dL1, dL2
+
+
 def max_err_vs_rms(got, ref) -> tuple[float, float]:
     """(max |got - ref|, RMS(ref)) in fp64: the tolerance test is max <= 2e-2 * RMS."""
     got, ref = _f64(got), _f64(ref)
