@@ -169,15 +169,36 @@ class Layer:
         B.qlora_linear_bwd(self.dY, self.X, self.p, self.L1, self.L2, self.s, sT=self.sT,
                            dX=self.dX, dL1=self.dL1, dL2=self.dL2, ws=self.wsb)
 
+    def step_dropout(self, p: float, seed: int):
+        """The same step with LoRA dropout on the adapter input (workspaces made on first use)."""
+        from bit_quantized_lora_03_b200 import binding as B
+        if not hasattr(self, "wsfd"):
+            dev = self.X.device
+            lib = B.lib()
+            self.wsfd = torch.empty(lib.qlora_fwd_dropout_workspace_bytes(self.t, self.h, self.o, self.r),
+                                    dtype=torch.uint8, device=dev)
+            self.wsbd = torch.empty(lib.qlora_bwd_dropout_workspace_bytes(self.t, self.h, self.o, self.r),
+                                    dtype=torch.uint8, device=dev)
+        B.qlora_linear_fwd_dropout(self.X, self.p, self.L1, self.L2, self.s, p, seed, Y=self.Y,
+                                   sT=self.sT, ws=self.wsfd)
+        B.qlora_linear_bwd_dropout(self.dY, self.X, self.p, self.L1, self.L2, self.s, p, seed,
+                                   sT=self.sT, dX=self.dX, dL1=self.dL1, dL2=self.dL2, ws=self.wsbd)
 
-def step_all(layers, world, streams=None):
-    """One step: fwd+bwd of every linear. The linears are independent, so with `streams` they
-    run round-robin on those streams (joined back to the caller's stream), letting one
-    linear's kernels fill the SMs another's last wave leaves idle."""
+    def free_dropout(self):
+        for k in ("wsfd", "wsbd"):
+            if hasattr(self, k):
+                delattr(self, k)
+
+
+def step_all(layers, world, streams=None, one=None):
+    """One step: fwd+bwd of every linear (`one(L)`, default L.step()). The linears are
+    independent, so with `streams` they run round-robin on those streams (joined back to the
+    caller's stream), letting one linear's kernels fill the SMs another's last wave leaves idle."""
     from bit_quantized_lora_03_b200 import dp
+    one = one or (lambda L: L.step())
     if not streams:
         for L in layers:
-            L.step()
+            one(L)
     else:
         cur = torch.cuda.current_stream()
         go = torch.cuda.Event()
@@ -186,7 +207,7 @@ def step_all(layers, world, streams=None):
             st.wait_event(go)
         for i, L in enumerate(layers):
             with torch.cuda.stream(streams[i % len(streams)]):
-                L.step()
+                one(L)
         for st in streams:
             done = torch.cuda.Event()
             done.record(st)
@@ -524,6 +545,42 @@ def merge_leg(dev, peaks, r: int = 64, s: float = 0.25):
     return res
 
 
+def dropout_leg(dev, peaks, layers, streams, base_ms_step, steps: int = 30, p: float = 0.05):
+    """The headline step with LoRA dropout p on every linear's adapter input (the mask drawn in
+    the kernels, a fresh seed per linear and step): tokens/s against the same step without
+    dropout, and the mask kernel's bandwidth (read 2 B + write 2 B per input element)."""
+    from bit_quantized_lora_03_b200 import binding as B
+    t = layers[0].t
+    counter = [0]
+
+    def one(L):
+        counter[0] += 1
+        L.step_dropout(p, 0xD00D_0000 + counter[0])
+    ms = timed(lambda: step_all(layers, 1, streams, one), steps, 3, 1, dev) / steps
+    with B.KernelProfile() as prof:
+        for _ in range(5):
+            step_all(layers, 1, None, one)
+    kname = "dropout_apply_kernel"
+    n_mask = prof.launches.get(kname, 0)
+    mask_ms = prof.ms.get(kname, 0.0) / max(1, n_mask)
+    # each linear's fwd and bwd apply the mask to its t x h input once
+    elems = sum(L.t * L.h for L in layers) * 2 * 5 / max(1, n_mask)
+    gbs = 4 * elems / (mask_ms * 1e-3) / 1e9 if mask_ms else None
+    tc_ms = prof.ms.get("tc_gemm_kernel", 0.0) / 5
+    res = {"p": p, "tokens_per_s": round(t / (ms * 1e-3), 1), "ms_per_step": round(ms, 4),
+           "vs_no_dropout_ms_per_step": round(base_ms_step, 4),
+           "overhead": round(ms / base_ms_step - 1.0, 4),
+           "mask_kernel_avg_ms": round(mask_ms, 4),
+           "mask_kernel_gbs": round(gbs, 1) if gbs else None,
+           "mask_kernel_frac_hbm": round(gbs / peaks["hbm_gbs"], 3) if gbs else None,
+           "tc_gemm_ms_per_step": round(tc_ms, 4),
+           "device_status": B.last_status()}
+    for L in layers:
+        L.free_dropout()
+    torch.cuda.empty_cache()
+    return res
+
+
 # ------------------------------------------------------------------------------------------
 # CPU oracle baseline (bounded sample)
 # ------------------------------------------------------------------------------------------
@@ -624,6 +681,8 @@ def main():
                     help="streams the 7 independent linears of a step are spread over")
     ap.add_argument("--single-linear", type=int, default=None, metavar="I",
                     help="profiling case: only linear I of the layer, fwd+bwd, no extras")
+    ap.add_argument("--dropout-only", action="store_true",
+                    help="after the headline, run only the LoRA-dropout leg (no other legs, no CPU baseline)")
     ap.add_argument("--decode-case", type=int, nargs=2, default=None, metavar=("T", "I"),
                     help="profiling case: quantize decode weight I, then three forward calls "
                          "at T tokens")
@@ -744,6 +803,9 @@ def main():
     legs = {}
     cpu = None
     if rank == 0 and world == 1 and not args.quick:
+        dstreams = [torch.cuda.Stream(dev) for _ in range(args.streams)] if args.streams > 1 else None
+        legs["dropout_llama7b_layer"] = dropout_leg(dev, peaks, layers, dstreams, ms_step)
+    if rank == 0 and world == 1 and not args.quick and not args.dropout_only:
         del layers
         torch.cuda.empty_cache()
         legs["decode_gemv"] = gemv_leg(dev, peaks, l2_bytes)

@@ -58,8 +58,18 @@ SIGNATURES = {
     "qlora_kernel_name": (ctypes.c_char_p, [ctypes.c_int]),
     "qlora_linear_fwd_noalloc": (ctypes.c_int, [_PTR, _I64, _PTR, _PTR, _PTR, _I64,
                                                 ctypes.c_float, _PTR, _PTR, _PTR]),
+    "qlora_linear_fwd_dropout": (ctypes.c_int, [_PTR, _I64, _PTR, _PTR, _PTR, _I64, ctypes.c_float,
+                                                ctypes.c_float, ctypes.c_uint64, _PTR, _PTR, _PTR,
+                                                ctypes.c_size_t, _PTR]),
+    "qlora_linear_bwd_dropout": (ctypes.c_int, [_PTR, _PTR, _I64, _PTR, _PTR, _PTR, _I64,
+                                                ctypes.c_float, ctypes.c_float, ctypes.c_uint64,
+                                                _PTR, _PTR, _PTR, _PTR, _PTR, ctypes.c_size_t, _PTR]),
+    "qlora_fwd_dropout_workspace_bytes": (ctypes.c_size_t, [_I64, _I64, _I64, _I64]),
+    "qlora_bwd_dropout_workspace_bytes": (ctypes.c_size_t, [_I64, _I64, _I64, _I64]),
+    "qlora_dropout_apply": (ctypes.c_int, [_PTR, _I64, _I64, ctypes.c_float, ctypes.c_uint64, _PTR,
+                                           _PTR]),
 }
-KERNEL_KINDS = 7
+KERNEL_KINDS = 8
 
 
 class NF4WeightDesc(ctypes.Structure):
@@ -264,6 +274,83 @@ def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, p: PackedNF4, L1: torch.
                                 dL1.data_ptr(), dL2.data_ptr(), ws.data_ptr(), ws.numel(),
                                 _stream(stream))
     _check(rc, "qlora_linear_bwd")
+    return dX, dL1, dL2
+
+
+def _dropout_args(dropout_p: float, seed: int):
+    p32 = float(dropout_p)
+    if not (0.0 <= p32 < 1.0):
+        raise ValueError("dropout probability must lie in [0, 1)")
+    return ctypes.c_float(p32), ctypes.c_uint64(int(seed) & 0xFFFFFFFFFFFFFFFF)
+
+
+def qlora_dropout_apply(X: torch.Tensor, dropout_p: float, seed: int,
+                        out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """X (.) M for the LoRA-dropout keep mask M of (dropout_p, seed); dropped elements are +0."""
+    t, h = X.shape
+    _require(X, torch.bfloat16, (t, h), "X")
+    out = torch.empty_like(X) if out is None else out
+    _require(out, torch.bfloat16, (t, h), "out")
+    pf, sd = _dropout_args(dropout_p, seed)
+    _check(lib().qlora_dropout_apply(X.data_ptr(), t, h, pf, sd, out.data_ptr(), _stream(stream)),
+           "qlora_dropout_apply")
+    return out
+
+
+def qlora_linear_fwd_dropout(X: torch.Tensor, p: PackedNF4, L1: torch.Tensor, L2: torch.Tensor,
+                             s: float, dropout_p: float, seed: int, Y: torch.Tensor | None = None,
+                             sT: torch.Tensor | None = None, want_sT: bool = True,
+                             ws: torch.Tensor | None = None, stream=None):
+    """Y = X.W' + s.((X (.) M / (1 - p)).L1).L2 with the keep mask M of (dropout_p, seed).
+    Returns (Y, sT or None)."""
+    t, h = X.shape
+    o, r = p.out_features, L1.shape[1]
+    _require(X, torch.bfloat16, (t, h), "X")
+    _require(L1, torch.bfloat16, (h, r), "L1")
+    _require(L2, torch.bfloat16, (r, o), "L2")
+    if h != p.in_features:
+        raise ValueError("X and W disagree on in_features")
+    Y = torch.empty(t, o, dtype=torch.bfloat16, device=X.device) if Y is None else Y
+    if sT is None and want_sT:
+        sT = torch.empty(t, r, dtype=torch.bfloat16, device=X.device)
+    if ws is None:
+        ws = workspace(int(lib().qlora_fwd_dropout_workspace_bytes(t, h, o, r)), X.device)
+    pf, sd = _dropout_args(dropout_p, seed)
+    d = p.desc()
+    rc = lib().qlora_linear_fwd_dropout(X.data_ptr(), t, ctypes.byref(d), L1.data_ptr(),
+                                        L2.data_ptr(), r, float(s), pf, sd, Y.data_ptr(), _ptr(sT),
+                                        ws.data_ptr(), ws.numel(), _stream(stream))
+    _check(rc, "qlora_linear_fwd_dropout")
+    return Y, sT
+
+
+def qlora_linear_bwd_dropout(dY: torch.Tensor, X: torch.Tensor, p: PackedNF4, L1: torch.Tensor,
+                             L2: torch.Tensor, s: float, dropout_p: float, seed: int,
+                             sT: torch.Tensor | None = None, dX: torch.Tensor | None = None,
+                             dL1: torch.Tensor | None = None, dL2: torch.Tensor | None = None,
+                             ws: torch.Tensor | None = None, stream=None):
+    """Gradients for qlora_linear_fwd_dropout with the same (dropout_p, seed)."""
+    t, h = X.shape
+    o, r = p.out_features, L1.shape[1]
+    _require(dY, torch.bfloat16, (t, o), "dY")
+    _require(X, torch.bfloat16, (t, h), "X")
+    _require(L1, torch.bfloat16, (h, r), "L1")
+    _require(L2, torch.bfloat16, (r, o), "L2")
+    if sT is not None:
+        _require(sT, torch.bfloat16, (t, r), "sT")
+    dev = X.device
+    dX = torch.empty(t, h, dtype=torch.bfloat16, device=dev) if dX is None else dX
+    dL1 = torch.empty(h, r, dtype=torch.float32, device=dev) if dL1 is None else dL1
+    dL2 = torch.empty(r, o, dtype=torch.float32, device=dev) if dL2 is None else dL2
+    if ws is None:
+        ws = workspace(int(lib().qlora_bwd_dropout_workspace_bytes(t, h, o, r)), dev)
+    pf, sd = _dropout_args(dropout_p, seed)
+    d = p.desc()
+    rc = lib().qlora_linear_bwd_dropout(dY.data_ptr(), X.data_ptr(), t, ctypes.byref(d),
+                                        L1.data_ptr(), L2.data_ptr(), r, float(s), pf, sd, _ptr(sT),
+                                        dX.data_ptr(), dL1.data_ptr(), dL2.data_ptr(),
+                                        ws.data_ptr(), ws.numel(), _stream(stream))
+    _check(rc, "qlora_linear_bwd_dropout")
     return dX, dL1, dL2
 
 

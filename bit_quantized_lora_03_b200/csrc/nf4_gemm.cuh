@@ -65,6 +65,8 @@ struct Nf4GemmArgs {
   int num_lkb;      // LoRA K-steps: ceil(r/64)
   uint16_t* out;    // M x N bf16, row stride N
   Nf4Table tab;
+  const uint16_t* addend;  // NULL, or M x N bf16 added to the accumulator before the rounding;
+                           // written by the previous kernel on the stream (waited for first)
 };
 
 // Wait for an mbarrier phase ignoring the abort flag (used only to drain in-flight copies
@@ -333,6 +335,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     const bool done = mbar_wait(acc_full, 0, abort_flag);
     tc_fence_after();
     if (done && !*abort_flag) {
+      if (args.addend) pdl_wait();
       const int acc = warp >> 2, quad = warp & 3;
       const int row = mrow + acc * 256 + quad * 32 + lane;
       const uint32_t lane_addr =
@@ -343,6 +346,18 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         tmem_ld_16(lane_addr + c * 16, v);
         tmem_ld_wait();
         if (row < args.M) {
+          const int64_t off = static_cast<int64_t>(row) * args.N + n0 + c * 16;
+          if (args.addend) {
+            const uint4* ad = reinterpret_cast<const uint4*>(args.addend + off);
+            const uint4 a0 = ad[0], a1 = ad[1];
+            const uint32_t w[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {  // word k: column 2k in the low half, 2k + 1 high
+              v[2 * k] = __float_as_uint(__uint_as_float(v[2 * k]) + __uint_as_float(w[k] << 16));
+              v[2 * k + 1] = __float_as_uint(__uint_as_float(v[2 * k + 1]) +
+                                             __uint_as_float(w[k] & 0xFFFF0000u));
+            }
+          }
           uint4 o0, o1;
           o0.x = pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1]));
           o0.y = pack_bf16x2(__uint_as_float(v[2]), __uint_as_float(v[3]));
@@ -352,8 +367,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
           o1.y = pack_bf16x2(__uint_as_float(v[10]), __uint_as_float(v[11]));
           o1.z = pack_bf16x2(__uint_as_float(v[12]), __uint_as_float(v[13]));
           o1.w = pack_bf16x2(__uint_as_float(v[14]), __uint_as_float(v[15]));
-          uint4* dst = reinterpret_cast<uint4*>(args.out + static_cast<int64_t>(row) * args.N +
-                                                n0 + c * 16);
+          uint4* dst = reinterpret_cast<uint4*>(args.out + off);
           dst[0] = o0;
           dst[1] = o1;
         }

@@ -19,6 +19,7 @@
 #include "nf4_gemm.cuh"
 #include "tc_gemm.cuh"
 #include "adamw.cuh"
+#include "dropout.cuh"
 #include "nf4_gemv.cuh"
 
 using namespace qlora;
@@ -217,12 +218,12 @@ int launch_status() {
 // ------------------------------------------------------------------------------------------
 namespace prof {
 enum Kind {
-  kQuant = 0, kDequant, kGemv, kGemvLoraDown, kTcGemm, kGemmFwd, kGemmBwd, kKinds
+  kQuant = 0, kDequant, kGemv, kGemvLoraDown, kTcGemm, kGemmFwd, kGemmBwd, kDropout, kKinds
 };
 const char* const kNames[kKinds] = {
     "nf4_quantize_kernel", "nf4_dequantize_kernel", "nf4_gemv_kernel",
     "gemv_lora_down_kernel", "tc_gemm_kernel",
-    "nf4_gemm_kernel<fwd>", "nf4_gemm_kernel<bwd>"};
+    "nf4_gemm_kernel<fwd>", "nf4_gemm_kernel<bwd>", "dropout_apply_kernel"};
 static_assert(kKinds == QLORA_KERNEL_KINDS, "kernel kinds");
 
 struct State {
@@ -413,7 +414,7 @@ template <bool A_MN, bool B_MN>
 int launch_tc_gemm(const CUtensorMap& mA, const CUtensorMap& mB, int64_t M, int64_t ncols,
                    const TcPlan& pl, float alpha, int mode, float* out32, int64_t ld,
                    uint16_t* o16a, uint16_t* o16b, int pdl, cudaStream_t st,
-                   const nf4_weight* merge_w = nullptr) {
+                   const nf4_weight* merge_w = nullptr, const uint8_t* keep_bits = nullptr) {
   TcGemmArgs a{};
   a.M = static_cast<int>(M);
   a.Ncols = static_cast<int>(ncols);
@@ -435,6 +436,7 @@ int launch_tc_gemm(const CUtensorMap& mA, const CUtensorMap& mB, int64_t M, int6
     a.s2 = merge_w->absmax_s2;
     a.tab = device_table();
   }
+  a.keep_bits = keep_bits;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>((ncols + pl.BNp - 1) / pl.BNp), static_cast<unsigned>(pl.mtiles),
                      static_cast<unsigned>(pl.splits));
@@ -523,6 +525,259 @@ int lora_down(const CUtensorMap& mA, const CUtensorMap& mB, int64_t t, int64_t K
 #endif
   return launch_tc_gemm<false, B_MN>(mA, mB, t, r, pl, s, kOutRoundBf16, nullptr, r, out16,
                                      out16b, kPdlNone, st);
+}
+
+// ------------------------------------------------------------------------------------------
+// the adapted linear layer
+// ------------------------------------------------------------------------------------------
+// Dropout on the adapter input: key of the generator and the drop threshold floor(p * 2^32).
+DropoutKey dropout_key(float p, uint64_t seed) {
+  DropoutKey k{};
+  k.k0 = static_cast<uint32_t>(seed);
+  k.k1 = static_cast<uint32_t>(seed >> 32);
+  k.thr = static_cast<uint32_t>(std::floor(static_cast<double>(p) * 4294967296.0));
+  return k;
+}
+
+bool valid_dropout_p(float p) { return std::isfinite(p) && p >= 0.0f && p < 1.0f; }
+
+// X (.) M, t x h bf16
+size_t dropout_region_bytes(int64_t t, int64_t h) { return align256(static_cast<size_t>(t) * h * 2); }
+// the keep mask as bits, t x h / 8 bytes
+size_t keep_bits_bytes(int64_t t, int64_t h) { return align256(static_cast<size_t>(t) * h / 8); }
+
+int launch_dropout_apply(const uint16_t* X, int64_t n, uint16_t* Xd, uint8_t* bits,
+                         const DropoutKey& key, int sms, cudaStream_t st) {
+  const int64_t n8 = n / 8;
+  const int64_t per_block = 256 * kDropUnroll;
+  const int64_t blocks = std::max<int64_t>(
+      1, std::min<int64_t>((n8 + per_block - 1) / per_block, static_cast<int64_t>(sms) * 8));
+  {
+    prof::Scope ps(prof::kDropout, st);
+    dropout_apply_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        reinterpret_cast<const uint4*>(X), reinterpret_cast<uint4*>(Xd), bits, n8, key);
+  }
+  return launch_status();
+}
+
+int check_fwd_args(const uint16_t* X, int64_t t, const nf4_weight* W, const uint16_t* L1,
+                   const uint16_t* L2, int64_t r, float s, const uint16_t* Y, const uint16_t* sT_out,
+                   const void* workspace) {
+  if (!X || !L1 || !L2 || !Y) return QLORA_ERR_INVALID_ARG;
+  if (!std::isfinite(s)) return QLORA_ERR_INVALID_ARG;
+  int rc = check_weight(W);
+  if (rc) return rc;
+  if ((rc = check_linear_shape(t, W->in_features, W->out_features, r))) return rc;
+  if (!aligned16(X) || !aligned16(L1) || !aligned16(L2) || !aligned16(Y) ||
+      (sT_out && !aligned16(sT_out)) || (workspace && !aligned16(workspace)))
+    return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+int check_bwd_args(const uint16_t* dY, const uint16_t* X, int64_t t, const nf4_weight* W,
+                   const uint16_t* L1, const uint16_t* L2, int64_t r, float s,
+                   const uint16_t* sT_saved, const uint16_t* dX, const float* dL1, const float* dL2,
+                   const void* workspace) {
+  if (!dY || !X || !L1 || !L2 || !dX || !dL1 || !dL2) return QLORA_ERR_INVALID_ARG;
+  if (!std::isfinite(s)) return QLORA_ERR_INVALID_ARG;
+  int rc = check_weight(W);
+  if (rc) return rc;
+  if ((rc = check_linear_shape(t, W->in_features, W->out_features, r))) return rc;
+  if (!aligned16(dY) || !aligned16(X) || !aligned16(L1) || !aligned16(L2) || !aligned16(dX) ||
+      !aligned16(dL1) || !aligned16(dL2) || (sT_saved && !aligned16(sT_saved)) ||
+      (workspace && !aligned16(workspace)))
+    return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+// Y = X.W' + bf16(s . Xl.L1).L2. Xl is the adapter branch's input: X itself, or X with the
+// dropout mask applied (s then carries the 1 / (1 - p)). Arguments already checked.
+int fwd_core(const uint16_t* X, const uint16_t* Xl, int64_t t, const nf4_weight* W,
+             const uint16_t* L1, const uint16_t* L2, int64_t r, float s, uint16_t* Y,
+             uint16_t* sT_out, void* workspace, cudaStream_t st) {
+  int dev, rc;
+  if ((rc = current_device(&dev))) return rc;
+  const int64_t h = W->in_features, o = W->out_features;
+  const int sms = sm_count(dev);
+  if (t <= kGemvMaxTokens) {
+    // partial sums of Xl.L1 (+ zeroed sums and counters), then the GEMV, which forms
+    // sT = bf16(s . Xl.L1) and finishes Y
+    GemvWs gw = carve_gemv(workspace, t, o, r);
+    {
+      prof::Scope ps(prof::kGemvLoraDown, st);
+      gemv_lora_down_kernel<<<gd::kCtas, gd::kThreads, gd::smem_bytes(static_cast<int>(t), static_cast<int>(r)), st>>>(
+          Xl, L1, gw.Tpart, gw.Y32, gw.cnt, h, o, static_cast<int>(t), static_cast<int>(r));
+    }
+    if ((rc = launch_status())) return rc;
+    GemvArgs ga{};
+    ga.codes = W->codes;
+    ga.q8 = W->absmax_q8;
+    ga.s2 = W->absmax_s2;
+    ga.X = X;
+    ga.Tpart = gw.Tpart;
+    ga.sT_out = sT_out;
+    ga.s = s;
+    ga.L2 = L2;
+    ga.Y = Y;
+    ga.Y32 = gw.Y32;
+    ga.tile_cnt = gw.cnt;
+    ga.h = h;
+    ga.o = o;
+    ga.t = static_cast<int>(t);
+    ga.r = static_cast<int>(r);
+    ga.tab = device_table();
+    // one CTA of 16 warps per SM (fewer when there are fewer units than warps, or capped)
+    const int64_t units = (o / gv::kTileRows) * ((h / 64 + 1) / 2);
+    int64_t ctas = std::min<int64_t>(sms, (units + gv::kWarps - 1) / gv::kWarps);
+    const int cap = g_gemv_max_ctas.load(std::memory_order_relaxed);
+    if (cap > 0) ctas = std::min<int64_t>(ctas, cap);
+    dim3 grid(static_cast<unsigned>(ctas));
+    // codes as 32-row x 64-byte boxes (one unit each)
+    CUtensorMap mC;
+    if (!make_map_2d(&mC, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, h / 2, o, h / 2, 64,
+                     gv::kTileRows, false))
+      return QLORA_ERR_CUDA;
+    {
+      // programmatic dependent launch: the GEMV's CTAs may start (table, first code loads)
+      // while the LoRA-down kernel runs; they wait for its results before using them
+      prof::Scope ps(prof::kGemv, st);
+      cudaLaunchConfig_t cfg{};
+      cfg.gridDim = grid;
+      cfg.blockDim = dim3(gv::kThreads);
+      cfg.dynamicSmemBytes = gv::smem_bytes();
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      const cudaError_t e = t <= 8 ? cudaLaunchKernelEx(&cfg, nf4_gemv_kernel<1>, ga, mC)
+                                   : cudaLaunchKernelEx(&cfg, nf4_gemv_kernel<2>, ga, mC);
+      if (e != cudaSuccess) return QLORA_ERR_CUDA;
+    }
+    return launch_status();
+  }
+
+  LoraWs ws = carve_lora(workspace, t, r);
+
+  // T = Xl . L1 (t x r), then sT = bf16(s . T)
+  CUtensorMap mXl, mL1;
+  if (!map_bf16(&mXl, Xl, h, t, 64, 128) || !map_bf16(&mL1, L1, r, h, 64, 64)) return QLORA_ERR_CUDA;
+  uint16_t* sT = ws.b16;
+  if ((rc = lora_down<true>(mXl, mL1, t, h, r, s, sT, sT_out, sms, st))) return rc;
+
+  // Y = X . W' + sT . L2
+  CUtensorMap mA, mP, mA2, mB2;
+  if (!map_bf16(&mA, X, h, t, 64, 128) ||
+      !make_map_2d(&mP, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, h / 2, o, h / 2, 32, tc::BNH, false) ||
+      !map_bf16(&mA2, sT, r, t, 64, 128) || !map_bf16(&mB2, L2, o, r, 64, 64))
+    return QLORA_ERR_CUDA;
+  Nf4GemmArgs ga{};
+  ga.q8 = W->absmax_q8;
+  ga.s2 = W->absmax_s2;
+  ga.h = h;
+  ga.M = static_cast<int>(t);
+  ga.N = static_cast<int>(o);
+  ga.num_kb = static_cast<int>(h / 64);
+  ga.num_lkb = static_cast<int>((r + 63) / 64);
+  ga.out = Y;
+  ga.tab = device_table();
+  return launch_nf4_gemm<false>(mA, mP, mA2, mB2, ga, t, o, st, prof::kGemmFwd);
+}
+
+// dX = dY.W'^T + M (.) (sU.L1^T), dL1 = Xl^T.sU, dL2 = sT^T.dY with sU = bf16(s . dY.L2^T) and
+// sT = bf16(s . Xl.L1) (or the forward's copy). Without dropout (keep_bits == NULL) Xl = X, M
+// is all ones and the LoRA term of dX is a K-step of the fused kernel. With dropout Xl = X (.) M
+// (computed into `xd`, t x h bf16, by the caller, with the mask as bits in keep_bits: bit
+// e mod 8 of byte e / 8), s carries the 1 / (1 - p), and the masked term
+// E = bf16(M (.) sU.L1^T) is made after dL1 has consumed Xl, into the same buffer; the fused
+// kernel adds E to its fp32 accumulator before its one rounding to bf16. Arguments already
+// checked.
+int bwd_core(const uint16_t* dY, const uint16_t* Xl, int64_t t, const nf4_weight* W,
+             const uint16_t* L1, const uint16_t* L2, int64_t r, float s,
+             const uint16_t* sT_saved, uint16_t* dX, float* dL1, float* dL2, void* workspace,
+             cudaStream_t st, const uint8_t* keep_bits, uint16_t* xd) {
+  int dev, rc;
+  if ((rc = current_device(&dev))) return rc;
+  const int64_t h = W->in_features, o = W->out_features;
+  const int sms = sm_count(dev);
+  LoraWs wsU = carve_lora(workspace, t, r);
+  LoraWs wsT = carve_lora(reinterpret_cast<uint8_t*>(workspace) + lora_region_bytes(t, r), t, r);
+
+  // sU = bf16(s . dY . L2^T): A = dY (t x o, K-major), B[k=j][n=c] = L2[c][j] (K-major)
+  CUtensorMap mdY, mL2k;
+  if (!map_bf16(&mdY, dY, o, t, 64, 128) ||
+      !map_bf16(&mL2k, L2, o, r, 64, static_cast<uint32_t>((r + 15) / 16 * 16)))
+    return QLORA_ERR_CUDA;
+  uint16_t* sU = wsU.b16;
+  if ((rc = lora_down<false>(mdY, mL2k, t, o, r, s, sU, nullptr, sms, st))) return rc;
+
+  // sT = bf16(s . Xl . L1) unless the forward's copy was passed in
+  const uint16_t* sT = sT_saved;
+  if (!sT) {
+    CUtensorMap mXl, mL1;
+    if (!map_bf16(&mXl, Xl, h, t, 64, 128) || !map_bf16(&mL1, L1, r, h, 64, 64)) return QLORA_ERR_CUDA;
+    if ((rc = lora_down<true>(mXl, mL1, t, h, r, s, wsT.b16, nullptr, sms, st))) return rc;
+    sT = wsT.b16;
+  }
+
+  // Launch order U [, sT], dL1, [E,] dX, dL2, each after the first by programmatic dependent
+  // launch: dL1 waits for sU; E waits for dL1 (it overwrites dL1's input); the fused dX kernel
+  // streams dY and W' while the kernel before it runs and waits for it (hence for sU, and for E)
+  // before its LoRA K-step or its epilogue; dL2 needs nothing made in this call unless sT was
+  // recomputed, so it can fill the SMs the dX kernel's last wave leaves idle.
+  // dL1 = Xl^T . sU (h x r) and dL2^T = dY^T . sT (o x r), reductions over the t tokens
+  CUtensorMap mXmn, msU, mdYmn, msT;
+  if (!map_bf16(&mXmn, Xl, h, t, 64, 64) || !map_bf16(&msU, sU, r, t, 64, 64) ||
+      !map_bf16(&mdYmn, dY, o, t, 64, 64) || !map_bf16(&msT, sT, r, t, 64, 64))
+    return QLORA_ERR_CUDA;
+  const TcPlan p1 = plan_tc(h, r, t, true, sms);
+  if ((rc = launch_tc_gemm<true, true>(mXmn, msU, h, r, p1, 1.0f, kOutRowMajor, dL1, r,
+                                       nullptr, nullptr, kPdlWaitFirst, st)))
+    return rc;
+
+  const uint16_t* E = nullptr;
+  if (keep_bits) {
+    // E = bf16(M (.) sU . L1^T), t x h: a K = r product (one CTA per 128 x BNp tile, no
+    // split-K) whose epilogue applies the keep bits
+    TcPlan pm = plan_tc(t, h, r, false, sms);
+    pm.splits = 1;
+    pm.kb_per_split = pm.num_kb;
+    pm.stages = std::max(2, std::min(pm.stages, pm.num_kb));
+    pm.smem = tcg::smem_bytes(pm.stages, pm.BNp, false);
+    CUtensorMap mU, mL1k;
+    if (!map_bf16(&mU, sU, r, t, 64, 128) || !map_bf16(&mL1k, L1, r, h, 64, static_cast<uint32_t>(pm.BNp)))
+      return QLORA_ERR_CUDA;
+    if ((rc = launch_tc_gemm<false, false>(mU, mL1k, t, h, pm, 1.0f, kOutMaskBf16, nullptr, h, xd,
+                                           nullptr, kPdlWaitFirst, st, nullptr, keep_bits)))
+      return rc;
+    E = xd;
+  }
+
+  // dX = dY . W'^T + sU . L1^T (one accumulator), or dY . W'^T + E
+  {
+    CUtensorMap mA, mP, mA2, mB2;
+    if (!map_bf16(&mA, dY, o, t, 64, 128) ||
+        !make_map_2d(&mP, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, h / 2, o, h / 2, 32, 64, false) ||
+        !map_bf16(&mA2, sU, r, t, 64, 128) || !map_bf16(&mB2, L1, r, h, 64, tc::BNH))
+      return QLORA_ERR_CUDA;
+    Nf4GemmArgs ga{};
+    ga.q8 = W->absmax_q8;
+    ga.s2 = W->absmax_s2;
+    ga.h = h;
+    ga.M = static_cast<int>(t);
+    ga.N = static_cast<int>(h);
+    ga.num_kb = static_cast<int>(o / 64);
+    ga.num_lkb = E ? 0 : static_cast<int>((r + 63) / 64);
+    ga.out = dX;
+    ga.tab = device_table();
+    ga.addend = E;
+    if ((rc = launch_nf4_gemm<true>(mA, mP, mA2, mB2, ga, t, h, st, prof::kGemmBwd))) return rc;
+  }
+
+  const TcPlan p2 = plan_tc(o, r, t, true, sms);
+  return launch_tc_gemm<true, true>(mdYmn, msT, o, r, p2, 1.0f, kOutTransposed, dL2, o, nullptr,
+                                    nullptr, sT_saved ? kPdlWaitLast : kPdlWaitFirst, st);
 }
 
 }  // namespace
@@ -803,184 +1058,93 @@ int qlora_codebook(int codebook_id, float* levels, float* midpoints) {
 int qlora_linear_fwd(const uint16_t* X, int64_t t, const nf4_weight* W, const uint16_t* L1,
                      const uint16_t* L2, int64_t r, float s, uint16_t* Y, uint16_t* sT_out,
                      void* workspace, size_t ws_bytes, qlora_stream_t stream) {
-  if (!X || !L1 || !L2 || !Y) return QLORA_ERR_INVALID_ARG;
-  if (!std::isfinite(s)) return QLORA_ERR_INVALID_ARG;
-  int rc = check_weight(W);
+  int rc = check_fwd_args(X, t, W, L1, L2, r, s, Y, sT_out, workspace);
   if (rc) return rc;
-  const int64_t h = W->in_features, o = W->out_features;
-  if ((rc = check_linear_shape(t, h, o, r))) return rc;
-  if (!aligned16(X) || !aligned16(L1) || !aligned16(L2) || !aligned16(Y) ||
-      (sT_out && !aligned16(sT_out)) || (workspace && !aligned16(workspace)))
-    return QLORA_ERR_MISALIGNED;
-  if (!workspace || ws_bytes < qlora_fwd_workspace_bytes(t, h, o, r)) return QLORA_ERR_WORKSPACE;
-  int dev;
-  if ((rc = current_device(&dev))) return rc;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int sms = sm_count(dev);
-  if (t <= kGemvMaxTokens) {
-    // partial sums of X.L1 (+ zeroed sums and counters), then the GEMV, which forms
-    // sT = bf16(s . X.L1) and finishes Y
-    GemvWs gw = carve_gemv(workspace, t, o, r);
-    {
-      prof::Scope ps(prof::kGemvLoraDown, st);
-      gemv_lora_down_kernel<<<gd::kCtas, gd::kThreads, gd::smem_bytes(static_cast<int>(t), static_cast<int>(r)), st>>>(
-          X, L1, gw.Tpart, gw.Y32, gw.cnt, h, o, static_cast<int>(t), static_cast<int>(r));
-    }
-    if ((rc = launch_status())) return rc;
-    GemvArgs ga{};
-    ga.codes = W->codes;
-    ga.q8 = W->absmax_q8;
-    ga.s2 = W->absmax_s2;
-    ga.X = X;
-    ga.Tpart = gw.Tpart;
-    ga.sT_out = sT_out;
-    ga.s = s;
-    ga.L2 = L2;
-    ga.Y = Y;
-    ga.Y32 = gw.Y32;
-    ga.tile_cnt = gw.cnt;
-    ga.h = h;
-    ga.o = o;
-    ga.t = static_cast<int>(t);
-    ga.r = static_cast<int>(r);
-    ga.tab = device_table();
-    // one CTA of 16 warps per SM (fewer when there are fewer units than warps, or capped)
-    const int64_t units = (o / gv::kTileRows) * ((h / 64 + 1) / 2);
-    int64_t ctas = std::min<int64_t>(sms, (units + gv::kWarps - 1) / gv::kWarps);
-    const int cap = g_gemv_max_ctas.load(std::memory_order_relaxed);
-    if (cap > 0) ctas = std::min<int64_t>(ctas, cap);
-    dim3 grid(static_cast<unsigned>(ctas));
-    // codes as 32-row x 64-byte boxes (one unit each)
-    CUtensorMap mC;
-    if (!make_map_2d(&mC, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, h / 2, o, h / 2, 64,
-                     gv::kTileRows, false))
-      return QLORA_ERR_CUDA;
-    {
-      // programmatic dependent launch: the GEMV's CTAs may start (table, first code loads)
-      // while the LoRA-down kernel runs; they wait for its results before using them
-      prof::Scope ps(prof::kGemv, st);
-      cudaLaunchConfig_t cfg{};
-      cfg.gridDim = grid;
-      cfg.blockDim = dim3(gv::kThreads);
-      cfg.dynamicSmemBytes = gv::smem_bytes();
-      cfg.stream = st;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-      attr[0].val.programmaticStreamSerializationAllowed = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      const cudaError_t e = t <= 8 ? cudaLaunchKernelEx(&cfg, nf4_gemv_kernel<1>, ga, mC)
-                                   : cudaLaunchKernelEx(&cfg, nf4_gemv_kernel<2>, ga, mC);
-      if (e != cudaSuccess) return QLORA_ERR_CUDA;
-    }
-    return launch_status();
-  }
-
-  LoraWs ws = carve_lora(workspace, t, r);
-
-  // T = X . L1 (t x r), then sT = bf16(s . T)
-  CUtensorMap mX, mL1;
-  if (!map_bf16(&mX, X, h, t, 64, 128) || !map_bf16(&mL1, L1, r, h, 64, 64)) return QLORA_ERR_CUDA;
-
-
-  uint16_t* sT = ws.b16;
-  if ((rc = lora_down<true>(mX, mL1, t, h, r, s, sT, sT_out, sms, st))) return rc;
-
-  // Y = X . W' + sT . L2
-  CUtensorMap mA, mP, mA2, mB2;
-  if (!map_bf16(&mA, X, h, t, 64, 128) ||
-      !make_map_2d(&mP, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, h / 2, o, h / 2, 32, tc::BNH, false) ||
-      !map_bf16(&mA2, sT, r, t, 64, 128) || !map_bf16(&mB2, L2, o, r, 64, 64))
-    return QLORA_ERR_CUDA;
-  Nf4GemmArgs ga{};
-  ga.q8 = W->absmax_q8;
-  ga.s2 = W->absmax_s2;
-  ga.h = h;
-  ga.M = static_cast<int>(t);
-  ga.N = static_cast<int>(o);
-  ga.num_kb = static_cast<int>(h / 64);
-  ga.num_lkb = static_cast<int>((r + 63) / 64);
-  ga.out = Y;
-  ga.tab = device_table();
-  return launch_nf4_gemm<false>(mA, mP, mA2, mB2, ga, t, o, st, prof::kGemmFwd);
+  if (!workspace || ws_bytes < qlora_fwd_workspace_bytes(t, W->in_features, W->out_features, r))
+    return QLORA_ERR_WORKSPACE;
+  return fwd_core(X, X, t, W, L1, L2, r, s, Y, sT_out, workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t t, const nf4_weight* W,
                      const uint16_t* L1, const uint16_t* L2, int64_t r, float s,
                      const uint16_t* sT_saved, uint16_t* dX, float* dL1, float* dL2,
                      void* workspace, size_t ws_bytes, qlora_stream_t stream) {
-  if (!dY || !X || !L1 || !L2 || !dX || !dL1 || !dL2) return QLORA_ERR_INVALID_ARG;
-  if (!std::isfinite(s)) return QLORA_ERR_INVALID_ARG;
-  int rc = check_weight(W);
+  int rc = check_bwd_args(dY, X, t, W, L1, L2, r, s, sT_saved, dX, dL1, dL2, workspace);
   if (rc) return rc;
-  const int64_t h = W->in_features, o = W->out_features;
-  if ((rc = check_linear_shape(t, h, o, r))) return rc;
-  if (!aligned16(dY) || !aligned16(X) || !aligned16(L1) || !aligned16(L2) || !aligned16(dX) ||
-      !aligned16(dL1) || !aligned16(dL2) || (sT_saved && !aligned16(sT_saved)) ||
-      (workspace && !aligned16(workspace)))
-    return QLORA_ERR_MISALIGNED;
-  if (!workspace || ws_bytes < qlora_bwd_workspace_bytes(t, h, o, r)) return QLORA_ERR_WORKSPACE;
+  if (!workspace || ws_bytes < qlora_bwd_workspace_bytes(t, W->in_features, W->out_features, r))
+    return QLORA_ERR_WORKSPACE;
+  return bwd_core(dY, X, t, W, L1, L2, r, s, sT_saved, dX, dL1, dL2, workspace,
+                  reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr);
+}
+
+size_t qlora_fwd_dropout_workspace_bytes(int64_t t, int64_t h, int64_t o, int64_t r) {
+  const size_t base = qlora_fwd_workspace_bytes(t, h, o, r);
+  return base ? dropout_region_bytes(t, h) + base : 0;
+}
+
+size_t qlora_bwd_dropout_workspace_bytes(int64_t t, int64_t h, int64_t o, int64_t r) {
+  const size_t base = qlora_bwd_workspace_bytes(t, h, o, r);
+  return base ? dropout_region_bytes(t, h) + keep_bits_bytes(t, h) + base : 0;
+}
+
+int qlora_dropout_apply(const uint16_t* X, int64_t t, int64_t h, float p, uint64_t seed,
+                        uint16_t* Xd, qlora_stream_t stream) {
+  if (!X || !Xd || !valid_dropout_p(p)) return QLORA_ERR_INVALID_ARG;
+  if (t < 1 || h < 64 || h % 64 != 0 || t >= kMaxDim || h >= kMaxDim) return QLORA_ERR_BAD_SHAPE;
+  if (!aligned16(X) || !aligned16(Xd)) return QLORA_ERR_MISALIGNED;
+  int dev, rc;
+  if ((rc = current_device(&dev))) return rc;
+  return launch_dropout_apply(X, t * h, Xd, nullptr, dropout_key(p, seed), sm_count(dev),
+                              reinterpret_cast<cudaStream_t>(stream));
+}
+
+int qlora_linear_fwd_dropout(const uint16_t* X, int64_t t, const nf4_weight* W, const uint16_t* L1,
+                             const uint16_t* L2, int64_t r, float s, float p, uint64_t seed,
+                             uint16_t* Y, uint16_t* sT_out, void* workspace, size_t ws_bytes,
+                             qlora_stream_t stream) {
+  int rc = check_fwd_args(X, t, W, L1, L2, r, s, Y, sT_out, workspace);
+  if (rc) return rc;
+  if (!valid_dropout_p(p)) return QLORA_ERR_INVALID_ARG;
+  const float s_eff = s / (1.0f - p);
+  if (!std::isfinite(s_eff)) return QLORA_ERR_INVALID_ARG;
+  const int64_t h = W->in_features;
+  if (!workspace || ws_bytes < qlora_fwd_dropout_workspace_bytes(t, h, W->out_features, r))
+    return QLORA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint16_t* Xd = reinterpret_cast<uint16_t*>(workspace);
+  void* rest = reinterpret_cast<uint8_t*>(workspace) + dropout_region_bytes(t, h);
+  const DropoutKey key = dropout_key(p, seed);
+  if (key.thr == 0) return fwd_core(X, X, t, W, L1, L2, r, s, Y, sT_out, rest, st);
   int dev;
   if ((rc = current_device(&dev))) return rc;
+  if ((rc = launch_dropout_apply(X, t * h, Xd, nullptr, key, sm_count(dev), st))) return rc;
+  return fwd_core(X, Xd, t, W, L1, L2, r, s_eff, Y, sT_out, rest, st);
+}
+
+int qlora_linear_bwd_dropout(const uint16_t* dY, const uint16_t* X, int64_t t, const nf4_weight* W,
+                             const uint16_t* L1, const uint16_t* L2, int64_t r, float s, float p,
+                             uint64_t seed, const uint16_t* sT_saved, uint16_t* dX, float* dL1,
+                             float* dL2, void* workspace, size_t ws_bytes, qlora_stream_t stream) {
+  int rc = check_bwd_args(dY, X, t, W, L1, L2, r, s, sT_saved, dX, dL1, dL2, workspace);
+  if (rc) return rc;
+  if (!valid_dropout_p(p)) return QLORA_ERR_INVALID_ARG;
+  const float s_eff = s / (1.0f - p);
+  if (!std::isfinite(s_eff)) return QLORA_ERR_INVALID_ARG;
+  const int64_t h = W->in_features;
+  if (!workspace || ws_bytes < qlora_bwd_dropout_workspace_bytes(t, h, W->out_features, r))
+    return QLORA_ERR_WORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int sms = sm_count(dev);
-  LoraWs wsU = carve_lora(workspace, t, r);
-  LoraWs wsT = carve_lora(reinterpret_cast<uint8_t*>(workspace) + lora_region_bytes(t, r), t, r);
-
-  // sU = bf16(s . dY . L2^T): A = dY (t x o, K-major), B[k=j][n=c] = L2[c][j] (K-major)
-  CUtensorMap mdY, mL2k;
-  if (!map_bf16(&mdY, dY, o, t, 64, 128) ||
-      !map_bf16(&mL2k, L2, o, r, 64, static_cast<uint32_t>((r + 15) / 16 * 16)))
-    return QLORA_ERR_CUDA;
-  uint16_t* sU = wsU.b16;
-  if ((rc = lora_down<false>(mdY, mL2k, t, o, r, s, sU, nullptr, sms, st))) return rc;
-
-  // sT = bf16(s . X . L1) unless the forward's copy was passed in
-  const uint16_t* sT = sT_saved;
-  if (!sT) {
-    CUtensorMap mX, mL1;
-    if (!map_bf16(&mX, X, h, t, 64, 128) || !map_bf16(&mL1, L1, r, h, 64, 64)) return QLORA_ERR_CUDA;
-    if ((rc = lora_down<true>(mX, mL1, t, h, r, s, wsT.b16, nullptr, sms, st))) return rc;
-    sT = wsT.b16;
-  }
-
-  // Launch order U [, sT], dL1, dX, dL2, each after the first by programmatic dependent
-  // launch: dL1 waits for sU; the fused dX kernel streams dY and W' while dL1 runs and waits
-  // for it (hence for sU) before its LoRA K-step; dL2 needs nothing made in this call unless
-  // sT was recomputed, so it can fill the SMs the dX kernel's last wave leaves idle.
-  // dL1 = X^T . sU (h x r) and dL2^T = dY^T . sT (o x r), reductions over the t tokens
-  CUtensorMap mXmn, msU, mdYmn, msT;
-  if (!map_bf16(&mXmn, X, h, t, 64, 64) || !map_bf16(&msU, sU, r, t, 64, 64) ||
-      !map_bf16(&mdYmn, dY, o, t, 64, 64) || !map_bf16(&msT, sT, r, t, 64, 64))
-    return QLORA_ERR_CUDA;
-  const TcPlan p1 = plan_tc(h, r, t, true, sms);
-  if ((rc = launch_tc_gemm<true, true>(mXmn, msU, h, r, p1, 1.0f, kOutRowMajor, dL1, r,
-                                       nullptr, nullptr, kPdlWaitFirst, st)))
-    return rc;
-
-  // dX = dY . W'^T + sU . L1^T
-  {
-    CUtensorMap mA, mP, mA2, mB2;
-    if (!map_bf16(&mA, dY, o, t, 64, 128) ||
-        !make_map_2d(&mP, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, h / 2, o, h / 2, 32, 64, false) ||
-        !map_bf16(&mA2, sU, r, t, 64, 128) || !map_bf16(&mB2, L1, r, h, 64, tc::BNH))
-      return QLORA_ERR_CUDA;
-    Nf4GemmArgs ga{};
-    ga.q8 = W->absmax_q8;
-    ga.s2 = W->absmax_s2;
-    ga.h = h;
-    ga.M = static_cast<int>(t);
-    ga.N = static_cast<int>(h);
-    ga.num_kb = static_cast<int>(o / 64);
-    ga.num_lkb = static_cast<int>((r + 63) / 64);
-    ga.out = dX;
-    ga.tab = device_table();
-    if ((rc = launch_nf4_gemm<true>(mA, mP, mA2, mB2, ga, t, h, st, prof::kGemmBwd))) return rc;
-  }
-
-  const TcPlan p2 = plan_tc(o, r, t, true, sms);
-  return launch_tc_gemm<true, true>(mdYmn, msT, o, r, p2, 1.0f, kOutTransposed, dL2, o, nullptr,
-                                    nullptr, sT_saved ? kPdlWaitLast : kPdlWaitFirst, st);
+  uint8_t* b = reinterpret_cast<uint8_t*>(workspace);
+  uint16_t* Xd = reinterpret_cast<uint16_t*>(b);
+  uint8_t* bits = b + dropout_region_bytes(t, h);
+  void* rest = bits + keep_bits_bytes(t, h);
+  const DropoutKey key = dropout_key(p, seed);
+  if (key.thr == 0)
+    return bwd_core(dY, X, t, W, L1, L2, r, s, sT_saved, dX, dL1, dL2, rest, st, nullptr, nullptr);
+  int dev;
+  if ((rc = current_device(&dev))) return rc;
+  if ((rc = launch_dropout_apply(X, t * h, Xd, bits, key, sm_count(dev), st))) return rc;
+  return bwd_core(dY, Xd, t, W, L1, L2, r, s_eff, sT_saved, dX, dL1, dL2, rest, st, bits, Xd);
 }
 
 }  // extern "C"

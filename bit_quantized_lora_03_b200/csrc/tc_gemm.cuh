@@ -42,6 +42,8 @@ enum TcOutMode : int {
   kOutRoundBf16 = 2,  // out16a[m * Ncols + n] = bf16(alpha * acc) (and out16b if set)
   kOutMergeNF4 = 3,   // out32[m * ld + n] = W'[m][n] + alpha * acc, W' the dequantized NF4
                       // row m (of ld = h weights) of the packed weight in the args
+  kOutMaskBf16 = 4,   // out16a[m * Ncols + n] = bf16(M[m][n] * alpha * acc), M the dropout keep
+                      // mask: bit (e mod 8) of keep_bits[e / 8], e = m * Ncols + n (no split-K)
 };
 
 // Split-K runs as a thread-block cluster of `splits` CTAs along grid z (at most 8): each CTA
@@ -76,6 +78,7 @@ struct TcGemmArgs {
   const uint8_t* q8;
   const float* s2;
   Nf4Table tab;
+  const uint8_t* keep_bits;  // kOutMaskBf16: the keep mask, one bit per element
 };
 
 #ifdef QLORA_TRACE
@@ -248,6 +251,19 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
           reinterpret_cast<uint4*>(args.out16b + off)[0] = o0;
           reinterpret_cast<uint4*>(args.out16b + off)[1] = o1;
         }
+      } else if (args.out_mode == kOutMaskBf16) {
+        // the element index row * Ncols + n0 is a multiple of 16 (n0 % 16 == 0, Ncols % 64 == 0)
+        const int64_t off = static_cast<int64_t>(row) * args.Ncols + n0;
+        const uint32_t keep = *reinterpret_cast<const uint16_t*>(args.keep_bits + off / 8);
+        const float a = args.alpha;
+        uint32_t o[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)  // word k: element 2k in the low half, 2k + 1 high
+          o[k] = pack_bf16x2(((keep >> (2 * k)) & 1u) ? a * __uint_as_float(v[2 * k]) : 0.f,
+                             ((keep >> (2 * k + 1)) & 1u) ? a * __uint_as_float(v[2 * k + 1]) : 0.f);
+        uint4* d = reinterpret_cast<uint4*>(args.out16a + off);
+        d[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        d[1] = make_uint4(o[4], o[5], o[6], o[7]);
       } else {
         float* dst = args.out32 + static_cast<int64_t>(row) * args.ld + n0;
 #pragma unroll

@@ -179,6 +179,48 @@ QLORA_API int qlora_linear_fwd_noalloc(const uint16_t *X, int64_t t, const nf4_w
 QLORA_API size_t qlora_fwd_workspace_bytes(int64_t t, int64_t h, int64_t o, int64_t r);
 QLORA_API size_t qlora_bwd_workspace_bytes(int64_t t, int64_t h, int64_t o, int64_t r);
 
+/* LoRA dropout on the adapter input ("QLoRA in LLMs" section 12, "Minimal QLoRA Setup with
+ * Hugging Face": the example configuration uses a LoRA dropout of 0.05). The pages do not say
+ * where it acts; these calls take the adapter branch's input, with inverted scaling:
+ *   Y = X.W' + s.((X (.) M / (1 - p)).L1).L2,
+ * and the matching gradients dX = dY.W'^T + M (.) (s / (1 - p)).(dY.L2^T).L1^T,
+ * dL1 = s.(X (.) M / (1 - p))^T.(dY.L2^T), dL2 = s.((X (.) M / (1 - p)).L1)^T.dY.
+ * M (t x h) is drawn, not stored: element e = i*h + j takes word e mod 4 of Philox4x32-10
+ * (Salmon et al., "Parallel Random Numbers: As Easy as 1, 2, 3", SC'11) at counter
+ * (lo32(e / 4), hi32(e / 4), 0, 0) under key (lo32(seed), hi32(seed)), and is kept when that
+ * word is >= floor(p * 2^32). The forward and the backward of one step must get the same
+ * (p, seed); a new seed per step and per layer gives fresh masks.
+ *   p     dropout probability, 0 <= p < 1 (else INVALID_ARG); p = 0 (or any p below 2^-32) is
+ *         exactly the plain layer.
+ *   seed  any 64-bit value.
+ * Every other argument is that of qlora_linear_fwd / qlora_linear_bwd, except the workspace,
+ * which is larger (it holds X (.) M, and in the backward also the mask as bits and then the
+ * masked adapter term of dX):
+ * qlora_fwd_dropout_workspace_bytes and qlora_bwd_dropout_workspace_bytes. The rounded
+ * s / (1 - p) (fp32) is the scale of sT and sU; sT_out / sT_saved carry
+ * bf16(s / (1 - p) . (X (.) M).L1). In the backward the masked term
+ * E = bf16(M (.) sU.L1^T) is added to the fp32 accumulator of dY.W'^T before dX's one
+ * rounding to bf16. */
+QLORA_API int qlora_linear_fwd_dropout(const uint16_t *X, int64_t t, const nf4_weight *W,
+                                       const uint16_t *L1, const uint16_t *L2, int64_t r, float s,
+                                       float p, uint64_t seed, uint16_t *Y, uint16_t *sT_out,
+                                       void *workspace, size_t ws_bytes, qlora_stream_t stream);
+QLORA_API int qlora_linear_bwd_dropout(const uint16_t *dY, const uint16_t *X, int64_t t,
+                                       const nf4_weight *W, const uint16_t *L1, const uint16_t *L2,
+                                       int64_t r, float s, float p, uint64_t seed,
+                                       const uint16_t *sT_saved, uint16_t *dX, float *dL1,
+                                       float *dL2, void *workspace, size_t ws_bytes,
+                                       qlora_stream_t stream);
+QLORA_API size_t qlora_fwd_dropout_workspace_bytes(int64_t t, int64_t h, int64_t o, int64_t r);
+QLORA_API size_t qlora_bwd_dropout_workspace_bytes(int64_t t, int64_t h, int64_t o, int64_t r);
+
+/* qlora_dropout_apply -- Xd = X (.) M for the mask above (dropped elements become +0; no
+ * 1 / (1 - p) scaling), so that the mask can be inspected on its own.
+ *   X, Xd  device bf16, t x h row-major (may not overlap unless equal).  h % 64 == 0.
+ * Errors: INVALID_ARG (NULL, p outside [0, 1)), BAD_SHAPE, MISALIGNED. */
+QLORA_API int qlora_dropout_apply(const uint16_t *X, int64_t t, int64_t h, float p, uint64_t seed,
+                                  uint16_t *Xd, qlora_stream_t stream);
+
 /* Synchronise `stream`, then return and clear the device status word of the current device:
  * 0, or an OR of QLORA_DEV_* bits, or QLORA_ERR_CUDA if the synchronisation failed. */
 QLORA_API int qlora_get_last_status(qlora_stream_t stream);
@@ -193,7 +235,7 @@ QLORA_API int qlora_get_last_status(qlora_stream_t stream);
  * or QLORA_ERR_INVALID_ARG if the profile overflowed its capacity. Kinds are numbered
  * 0 .. QLORA_KERNEL_KINDS-1 and named by qlora_kernel_name. Not thread-safe across
  * concurrent calls into the library while open. */
-#define QLORA_KERNEL_KINDS 7
+#define QLORA_KERNEL_KINDS 8
 QLORA_API int qlora_profile_begin(int capacity);
 QLORA_API int qlora_profile_end(double *ms, int64_t *launches, int nkinds);
 QLORA_API const char *qlora_kernel_name(int kind);

@@ -140,3 +140,38 @@ def test_adamw_argument_checks(lib):
     assert call(lr=float("nan")) == B.QLORA_ERR_INVALID_ARG
     assert call(ptr=None) == B.QLORA_ERR_INVALID_ARG
     assert call(ptr=ctypes.c_void_p(20)) == B.QLORA_ERR_MISALIGNED
+
+
+def test_dropout_workspace_and_argument_checks(lib):
+    # the dropout calls hold X (.) M (t x h bf16), and the backward also the mask as bits,
+    # in front of the plain workspace
+    for t, h, o, r in ((4096, 4096, 11008, 64), (5, 320, 576, 16), (300, 640, 320, 48)):
+        xd = (t * h * 2 + 255) // 256 * 256
+        assert lib.qlora_fwd_dropout_workspace_bytes(t, h, o, r) == xd + lib.qlora_fwd_workspace_bytes(t, h, o, r)
+        bits = (t * h // 8 + 255) // 256 * 256
+        assert lib.qlora_bwd_dropout_workspace_bytes(t, h, o, r) == xd + bits + lib.qlora_bwd_workspace_bytes(t, h, o, r)
+    assert lib.qlora_fwd_dropout_workspace_bytes(8, 100, 4096, 64) == 0
+    assert lib.qlora_bwd_dropout_workspace_bytes(8, 4096, 4096, 512) == 0
+
+    d = _desc()
+    P = 0x10000
+    big = 1 << 30
+    fwd = lib.qlora_linear_fwd_dropout
+    for p in (-0.1, 1.0, 2.0, float("nan"), float("inf")):
+        assert fwd(P, 4, ctypes.byref(d), P, P, 16, 1.0, p, 1, P, None, P, big, None) == B.QLORA_ERR_INVALID_ARG
+    # s / (1 - p) must stay finite
+    assert fwd(P, 4, ctypes.byref(d), P, P, 16, 3e38, 0.5, 1, P, None, P, big, None) == B.QLORA_ERR_INVALID_ARG
+    assert fwd(P, 4, ctypes.byref(d), P, P, 16, 1.0, 0.1, 1, P, None, P, 1024, None) == B.QLORA_ERR_WORKSPACE
+    assert fwd(P + 2, 4, ctypes.byref(d), P, P, 16, 1.0, 0.1, 1, P, None, P, big, None) == B.QLORA_ERR_MISALIGNED
+    bwd = lib.qlora_linear_bwd_dropout
+    assert bwd(P, P, 4, ctypes.byref(d), P, P, 16, 1.0, 1.0, 1, None, P, P, P, P, big, None) == B.QLORA_ERR_INVALID_ARG
+    assert bwd(P, P, 4, ctypes.byref(d), P, P, 16, 1.0, 0.1, 1, None, P, P, None, P, big, None) == B.QLORA_ERR_INVALID_ARG
+    assert bwd(P, P, 4, ctypes.byref(d), P, P, 16, 1.0, 0.1, 1, None, P, P, P, P, 8, None) == B.QLORA_ERR_WORKSPACE
+    app = lib.qlora_dropout_apply
+    assert app(None, 4, 128, 0.1, 1, P, None) == B.QLORA_ERR_INVALID_ARG
+    assert app(P, 4, 128, 1.0, 1, P, None) == B.QLORA_ERR_INVALID_ARG
+    assert app(P, 4, 100, 0.1, 1, P, None) == B.QLORA_ERR_BAD_SHAPE
+    assert app(P, 0, 128, 0.1, 1, P, None) == B.QLORA_ERR_BAD_SHAPE
+    assert app(P, 4, 128, 0.1, 1, P + 8, None) == B.QLORA_ERR_MISALIGNED
+    with pytest.raises(ValueError):
+        B._dropout_args(1.0, 0)
