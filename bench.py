@@ -179,13 +179,15 @@ class Layer:
                                     dtype=torch.uint8, device=dev)
             self.wsbd = torch.empty(lib.qlora_bwd_dropout_workspace_bytes(self.t, self.h, self.o, self.r),
                                     dtype=torch.uint8, device=dev)
+            self.mask = torch.empty(B.dropout_mask_bytes(self.t, self.h), dtype=torch.uint8, device=dev)
         B.qlora_linear_fwd_dropout(self.X, self.p, self.L1, self.L2, self.s, p, seed, Y=self.Y,
-                                   sT=self.sT, ws=self.wsfd)
+                                   sT=self.sT, mask=self.mask, ws=self.wsfd)
         B.qlora_linear_bwd_dropout(self.dY, self.X, self.p, self.L1, self.L2, self.s, p, seed,
-                                   sT=self.sT, dX=self.dX, dL1=self.dL1, dL2=self.dL2, ws=self.wsbd)
+                                   sT=self.sT, mask=self.mask, dX=self.dX, dL1=self.dL1,
+                                   dL2=self.dL2, ws=self.wsbd)
 
     def free_dropout(self):
-        for k in ("wsfd", "wsbd"):
+        for k in ("wsfd", "wsbd", "mask"):
             if hasattr(self, k):
                 delattr(self, k)
 
@@ -547,8 +549,9 @@ def merge_leg(dev, peaks, r: int = 64, s: float = 0.25):
 
 def dropout_leg(dev, peaks, layers, streams, base_ms_step, steps: int = 30, p: float = 0.05):
     """The headline step with LoRA dropout p on every linear's adapter input (the mask drawn in
-    the kernels, a fresh seed per linear and step): tokens/s against the same step without
-    dropout, and the mask kernel's bandwidth (read 2 B + write 2 B per input element)."""
+    the forward's kernels, a fresh seed per linear and step, and handed to the backward as
+    bits): tokens/s against the same step without dropout, and the mask kernels' bandwidth
+    (read 2 B + write 2 B per input element, + 1/8 B of mask bits)."""
     from bit_quantized_lora_03_b200 import binding as B
     t = layers[0].t
     counter = [0]
@@ -565,7 +568,7 @@ def dropout_leg(dev, peaks, layers, streams, base_ms_step, steps: int = 30, p: f
     mask_ms = prof.ms.get(kname, 0.0) / max(1, n_mask)
     # each linear's fwd and bwd apply the mask to its t x h input once
     elems = sum(L.t * L.h for L in layers) * 2 * 5 / max(1, n_mask)
-    gbs = 4 * elems / (mask_ms * 1e-3) / 1e9 if mask_ms else None
+    gbs = 4.125 * elems / (mask_ms * 1e-3) / 1e9 if mask_ms else None
     tc_ms = prof.ms.get("tc_gemm_kernel", 0.0) / 5
     res = {"p": p, "tokens_per_s": round(t / (ms * 1e-3), 1), "ms_per_step": round(ms, 4),
            "vs_no_dropout_ms_per_step": round(base_ms_step, 4),
@@ -681,6 +684,8 @@ def main():
                     help="streams the 7 independent linears of a step are spread over")
     ap.add_argument("--single-linear", type=int, default=None, metavar="I",
                     help="profiling case: only linear I of the layer, fwd+bwd, no extras")
+    ap.add_argument("--dropout", type=float, default=0.0, metavar="P",
+                    help="with --single-linear: LoRA dropout P on the adapter input")
     ap.add_argument("--dropout-only", action="store_true",
                     help="after the headline, run only the LoRA-dropout leg (no other legs, no CPU baseline)")
     ap.add_argument("--decode-case", type=int, nargs=2, default=None, metavar=("T", "I"),
@@ -712,8 +717,10 @@ def main():
     t, r, s = args.tokens, 64, 0.25
     if args.single_linear is not None:
         L = Layer(args.single_linear, dev, t, r, s)
-        ms = timed(L.step, args.steps, args.warmup, 1, dev)
-        print(json.dumps({"case": f"single linear {L.name} h={L.h} o={L.o} t={t} r={r}",
+        fn = (lambda: L.step_dropout(args.dropout, 1234)) if args.dropout > 0 else L.step
+        ms = timed(fn, args.steps, args.warmup, 1, dev)
+        print(json.dumps({"case": f"single linear {L.name} h={L.h} o={L.o} t={t} r={r} "
+                                  f"dropout={args.dropout}",
                           "ms_per_fwd_bwd": round(ms / args.steps, 4),
                           "tflops": round(step_flops([L]) * args.steps / (ms * 1e-3) / 1e12, 1),
                           "device_status": B.last_status()}), flush=True)

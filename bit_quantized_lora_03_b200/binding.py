@@ -60,10 +60,11 @@ SIGNATURES = {
                                                 ctypes.c_float, _PTR, _PTR, _PTR]),
     "qlora_linear_fwd_dropout": (ctypes.c_int, [_PTR, _I64, _PTR, _PTR, _PTR, _I64, ctypes.c_float,
                                                 ctypes.c_float, ctypes.c_uint64, _PTR, _PTR, _PTR,
-                                                ctypes.c_size_t, _PTR]),
+                                                _PTR, ctypes.c_size_t, _PTR]),
     "qlora_linear_bwd_dropout": (ctypes.c_int, [_PTR, _PTR, _I64, _PTR, _PTR, _PTR, _I64,
                                                 ctypes.c_float, ctypes.c_float, ctypes.c_uint64,
-                                                _PTR, _PTR, _PTR, _PTR, _PTR, ctypes.c_size_t, _PTR]),
+                                                _PTR, _PTR, _PTR, _PTR, _PTR, _PTR, ctypes.c_size_t,
+                                                _PTR]),
     "qlora_fwd_dropout_workspace_bytes": (ctypes.c_size_t, [_I64, _I64, _I64, _I64]),
     "qlora_bwd_dropout_workspace_bytes": (ctypes.c_size_t, [_I64, _I64, _I64, _I64]),
     "qlora_dropout_apply": (ctypes.c_int, [_PTR, _I64, _I64, ctypes.c_float, ctypes.c_uint64, _PTR,
@@ -297,12 +298,19 @@ def qlora_dropout_apply(X: torch.Tensor, dropout_p: float, seed: int,
     return out
 
 
+def dropout_mask_bytes(t: int, h: int) -> int:
+    """Bytes of a keep mask stored as bits (bit e mod 8 of byte e / 8)."""
+    return t * h // 8
+
+
 def qlora_linear_fwd_dropout(X: torch.Tensor, p: PackedNF4, L1: torch.Tensor, L2: torch.Tensor,
                              s: float, dropout_p: float, seed: int, Y: torch.Tensor | None = None,
                              sT: torch.Tensor | None = None, want_sT: bool = True,
+                             mask: torch.Tensor | None = None, want_mask: bool = False,
                              ws: torch.Tensor | None = None, stream=None):
     """Y = X.W' + s.((X (.) M / (1 - p)).L1).L2 with the keep mask M of (dropout_p, seed).
-    Returns (Y, sT or None)."""
+    Returns (Y, sT or None, mask bits or None); pass the mask to the backward to spare it the
+    generator calls."""
     t, h = X.shape
     o, r = p.out_features, L1.shape[1]
     _require(X, torch.bfloat16, (t, h), "X")
@@ -313,23 +321,29 @@ def qlora_linear_fwd_dropout(X: torch.Tensor, p: PackedNF4, L1: torch.Tensor, L2
     Y = torch.empty(t, o, dtype=torch.bfloat16, device=X.device) if Y is None else Y
     if sT is None and want_sT:
         sT = torch.empty(t, r, dtype=torch.bfloat16, device=X.device)
+    if mask is None and want_mask:
+        mask = torch.empty(dropout_mask_bytes(t, h), dtype=torch.uint8, device=X.device)
+    if mask is not None:
+        _require(mask, torch.uint8, (dropout_mask_bytes(t, h),), "mask")
     if ws is None:
         ws = workspace(int(lib().qlora_fwd_dropout_workspace_bytes(t, h, o, r)), X.device)
     pf, sd = _dropout_args(dropout_p, seed)
     d = p.desc()
     rc = lib().qlora_linear_fwd_dropout(X.data_ptr(), t, ctypes.byref(d), L1.data_ptr(),
                                         L2.data_ptr(), r, float(s), pf, sd, Y.data_ptr(), _ptr(sT),
-                                        ws.data_ptr(), ws.numel(), _stream(stream))
+                                        _ptr(mask), ws.data_ptr(), ws.numel(), _stream(stream))
     _check(rc, "qlora_linear_fwd_dropout")
-    return Y, sT
+    return Y, sT, mask
 
 
 def qlora_linear_bwd_dropout(dY: torch.Tensor, X: torch.Tensor, p: PackedNF4, L1: torch.Tensor,
                              L2: torch.Tensor, s: float, dropout_p: float, seed: int,
-                             sT: torch.Tensor | None = None, dX: torch.Tensor | None = None,
+                             sT: torch.Tensor | None = None, mask: torch.Tensor | None = None,
+                             dX: torch.Tensor | None = None,
                              dL1: torch.Tensor | None = None, dL2: torch.Tensor | None = None,
                              ws: torch.Tensor | None = None, stream=None):
-    """Gradients for qlora_linear_fwd_dropout with the same (dropout_p, seed)."""
+    """Gradients for qlora_linear_fwd_dropout with the same (dropout_p, seed) (and, optionally,
+    the forward's mask bits)."""
     t, h = X.shape
     o, r = p.out_features, L1.shape[1]
     _require(dY, torch.bfloat16, (t, o), "dY")
@@ -338,6 +352,8 @@ def qlora_linear_bwd_dropout(dY: torch.Tensor, X: torch.Tensor, p: PackedNF4, L1
     _require(L2, torch.bfloat16, (r, o), "L2")
     if sT is not None:
         _require(sT, torch.bfloat16, (t, r), "sT")
+    if mask is not None:
+        _require(mask, torch.uint8, (dropout_mask_bytes(t, h),), "mask")
     dev = X.device
     dX = torch.empty(t, h, dtype=torch.bfloat16, device=dev) if dX is None else dX
     dL1 = torch.empty(h, r, dtype=torch.float32, device=dev) if dL1 is None else dL1
@@ -348,7 +364,7 @@ def qlora_linear_bwd_dropout(dY: torch.Tensor, X: torch.Tensor, p: PackedNF4, L1
     d = p.desc()
     rc = lib().qlora_linear_bwd_dropout(dY.data_ptr(), X.data_ptr(), t, ctypes.byref(d),
                                         L1.data_ptr(), L2.data_ptr(), r, float(s), pf, sd, _ptr(sT),
-                                        dX.data_ptr(), dL1.data_ptr(), dL2.data_ptr(),
+                                        _ptr(mask), dX.data_ptr(), dL1.data_ptr(), dL2.data_ptr(),
                                         ws.data_ptr(), ws.numel(), _stream(stream))
     _check(rc, "qlora_linear_bwd_dropout")
     return dX, dL1, dL2

@@ -546,7 +546,9 @@ size_t dropout_region_bytes(int64_t t, int64_t h) { return align256(static_cast<
 // the keep mask as bits, t x h / 8 bytes
 size_t keep_bits_bytes(int64_t t, int64_t h) { return align256(static_cast<size_t>(t) * h / 8); }
 
-int launch_dropout_apply(const uint16_t* X, int64_t n, uint16_t* Xd, uint8_t* bits,
+// Xd = X (.) M; the keep bits are drawn (and stored into `bits` if given) or, with from_bits,
+// read from `bits`.
+int launch_dropout_apply(const uint16_t* X, int64_t n, uint16_t* Xd, uint8_t* bits, bool from_bits,
                          const DropoutKey& key, int sms, cudaStream_t st) {
   const int64_t n8 = n / 8;
   const int64_t per_block = 256 * kDropUnroll;
@@ -554,7 +556,8 @@ int launch_dropout_apply(const uint16_t* X, int64_t n, uint16_t* Xd, uint8_t* bi
       1, std::min<int64_t>((n8 + per_block - 1) / per_block, static_cast<int64_t>(sms) * 8));
   {
     prof::Scope ps(prof::kDropout, st);
-    dropout_apply_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+    const auto kern = from_bits ? dropout_apply_kernel<true> : dropout_apply_kernel<false>;
+    kern<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
         reinterpret_cast<const uint4*>(X), reinterpret_cast<uint4*>(Xd), bits, n8, key);
   }
   return launch_status();
@@ -1094,19 +1097,20 @@ int qlora_dropout_apply(const uint16_t* X, int64_t t, int64_t h, float p, uint64
   if (!aligned16(X) || !aligned16(Xd)) return QLORA_ERR_MISALIGNED;
   int dev, rc;
   if ((rc = current_device(&dev))) return rc;
-  return launch_dropout_apply(X, t * h, Xd, nullptr, dropout_key(p, seed), sm_count(dev),
+  return launch_dropout_apply(X, t * h, Xd, nullptr, false, dropout_key(p, seed), sm_count(dev),
                               reinterpret_cast<cudaStream_t>(stream));
 }
 
 int qlora_linear_fwd_dropout(const uint16_t* X, int64_t t, const nf4_weight* W, const uint16_t* L1,
                              const uint16_t* L2, int64_t r, float s, float p, uint64_t seed,
-                             uint16_t* Y, uint16_t* sT_out, void* workspace, size_t ws_bytes,
-                             qlora_stream_t stream) {
+                             uint16_t* Y, uint16_t* sT_out, uint8_t* mask_out, void* workspace,
+                             size_t ws_bytes, qlora_stream_t stream) {
   int rc = check_fwd_args(X, t, W, L1, L2, r, s, Y, sT_out, workspace);
   if (rc) return rc;
   if (!valid_dropout_p(p)) return QLORA_ERR_INVALID_ARG;
   const float s_eff = s / (1.0f - p);
   if (!std::isfinite(s_eff)) return QLORA_ERR_INVALID_ARG;
+  if (mask_out && !aligned16(mask_out)) return QLORA_ERR_MISALIGNED;
   const int64_t h = W->in_features;
   if (!workspace || ws_bytes < qlora_fwd_dropout_workspace_bytes(t, h, W->out_features, r))
     return QLORA_ERR_WORKSPACE;
@@ -1114,22 +1118,30 @@ int qlora_linear_fwd_dropout(const uint16_t* X, int64_t t, const nf4_weight* W, 
   uint16_t* Xd = reinterpret_cast<uint16_t*>(workspace);
   void* rest = reinterpret_cast<uint8_t*>(workspace) + dropout_region_bytes(t, h);
   const DropoutKey key = dropout_key(p, seed);
-  if (key.thr == 0) return fwd_core(X, X, t, W, L1, L2, r, s, Y, sT_out, rest, st);
+  if (key.thr == 0) {
+    if (mask_out && cudaMemsetAsync(mask_out, 0xFF, static_cast<size_t>(t) * h / 8, st) != cudaSuccess) {
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
+    return fwd_core(X, X, t, W, L1, L2, r, s, Y, sT_out, rest, st);
+  }
   int dev;
   if ((rc = current_device(&dev))) return rc;
-  if ((rc = launch_dropout_apply(X, t * h, Xd, nullptr, key, sm_count(dev), st))) return rc;
+  if ((rc = launch_dropout_apply(X, t * h, Xd, mask_out, false, key, sm_count(dev), st))) return rc;
   return fwd_core(X, Xd, t, W, L1, L2, r, s_eff, Y, sT_out, rest, st);
 }
 
 int qlora_linear_bwd_dropout(const uint16_t* dY, const uint16_t* X, int64_t t, const nf4_weight* W,
                              const uint16_t* L1, const uint16_t* L2, int64_t r, float s, float p,
-                             uint64_t seed, const uint16_t* sT_saved, uint16_t* dX, float* dL1,
-                             float* dL2, void* workspace, size_t ws_bytes, qlora_stream_t stream) {
+                             uint64_t seed, const uint16_t* sT_saved, const uint8_t* mask_saved,
+                             uint16_t* dX, float* dL1, float* dL2, void* workspace, size_t ws_bytes,
+                             qlora_stream_t stream) {
   int rc = check_bwd_args(dY, X, t, W, L1, L2, r, s, sT_saved, dX, dL1, dL2, workspace);
   if (rc) return rc;
   if (!valid_dropout_p(p)) return QLORA_ERR_INVALID_ARG;
   const float s_eff = s / (1.0f - p);
   if (!std::isfinite(s_eff)) return QLORA_ERR_INVALID_ARG;
+  if (mask_saved && !aligned16(mask_saved)) return QLORA_ERR_MISALIGNED;
   const int64_t h = W->in_features;
   if (!workspace || ws_bytes < qlora_bwd_dropout_workspace_bytes(t, h, W->out_features, r))
     return QLORA_ERR_WORKSPACE;
@@ -1143,8 +1155,11 @@ int qlora_linear_bwd_dropout(const uint16_t* dY, const uint16_t* X, int64_t t, c
     return bwd_core(dY, X, t, W, L1, L2, r, s, sT_saved, dX, dL1, dL2, rest, st, nullptr, nullptr);
   int dev;
   if ((rc = current_device(&dev))) return rc;
-  if ((rc = launch_dropout_apply(X, t * h, Xd, bits, key, sm_count(dev), st))) return rc;
-  return bwd_core(dY, Xd, t, W, L1, L2, r, s_eff, sT_saved, dX, dL1, dL2, rest, st, bits, Xd);
+  // the forward's mask when given (no generator calls), else drawn again from (p, seed)
+  uint8_t* mask = mask_saved ? const_cast<uint8_t*>(mask_saved) : bits;
+  if ((rc = launch_dropout_apply(X, t * h, Xd, mask, mask_saved != nullptr, key, sm_count(dev), st)))
+    return rc;
+  return bwd_core(dY, Xd, t, W, L1, L2, r, s_eff, sT_saved, dX, dL1, dL2, rest, st, mask, Xd);
 }
 
 }  // extern "C"

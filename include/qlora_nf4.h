@@ -193,6 +193,10 @@ QLORA_API size_t qlora_bwd_workspace_bytes(int64_t t, int64_t h, int64_t o, int6
  *   p     dropout probability, 0 <= p < 1 (else INVALID_ARG); p = 0 (or any p below 2^-32) is
  *         exactly the plain layer.
  *   seed  any 64-bit value.
+ *   mask_out    (forward) device, t*h/8 bytes, 16-byte aligned, or NULL: receives M as bits,
+ *               bit e mod 8 of byte e / 8 = keep bit of element e.
+ *   mask_saved  (backward) the forward's mask_out for the same (p, seed), or NULL to draw M
+ *               again; with it the backward makes no generator calls.
  * Every other argument is that of qlora_linear_fwd / qlora_linear_bwd, except the workspace,
  * which is larger (it holds X (.) M, and in the backward also the mask as bits and then the
  * masked adapter term of dX):
@@ -204,13 +208,14 @@ QLORA_API size_t qlora_bwd_workspace_bytes(int64_t t, int64_t h, int64_t o, int6
 QLORA_API int qlora_linear_fwd_dropout(const uint16_t *X, int64_t t, const nf4_weight *W,
                                        const uint16_t *L1, const uint16_t *L2, int64_t r, float s,
                                        float p, uint64_t seed, uint16_t *Y, uint16_t *sT_out,
-                                       void *workspace, size_t ws_bytes, qlora_stream_t stream);
+                                       uint8_t *mask_out, void *workspace, size_t ws_bytes,
+                                       qlora_stream_t stream);
 QLORA_API int qlora_linear_bwd_dropout(const uint16_t *dY, const uint16_t *X, int64_t t,
                                        const nf4_weight *W, const uint16_t *L1, const uint16_t *L2,
                                        int64_t r, float s, float p, uint64_t seed,
-                                       const uint16_t *sT_saved, uint16_t *dX, float *dL1,
-                                       float *dL2, void *workspace, size_t ws_bytes,
-                                       qlora_stream_t stream);
+                                       const uint16_t *sT_saved, const uint8_t *mask_saved,
+                                       uint16_t *dX, float *dL1, float *dL2, void *workspace,
+                                       size_t ws_bytes, qlora_stream_t stream);
 QLORA_API size_t qlora_fwd_dropout_workspace_bytes(int64_t t, int64_t h, int64_t o, int64_t r);
 QLORA_API size_t qlora_bwd_dropout_workspace_bytes(int64_t t, int64_t h, int64_t o, int64_t r);
 

@@ -158,15 +158,18 @@ def test_dropout_workspace_and_argument_checks(lib):
     big = 1 << 30
     fwd = lib.qlora_linear_fwd_dropout
     for p in (-0.1, 1.0, 2.0, float("nan"), float("inf")):
-        assert fwd(P, 4, ctypes.byref(d), P, P, 16, 1.0, p, 1, P, None, P, big, None) == B.QLORA_ERR_INVALID_ARG
+        assert fwd(P, 4, ctypes.byref(d), P, P, 16, 1.0, p, 1, P, None, None, P, big, None) == B.QLORA_ERR_INVALID_ARG
     # s / (1 - p) must stay finite
-    assert fwd(P, 4, ctypes.byref(d), P, P, 16, 3e38, 0.5, 1, P, None, P, big, None) == B.QLORA_ERR_INVALID_ARG
-    assert fwd(P, 4, ctypes.byref(d), P, P, 16, 1.0, 0.1, 1, P, None, P, 1024, None) == B.QLORA_ERR_WORKSPACE
-    assert fwd(P + 2, 4, ctypes.byref(d), P, P, 16, 1.0, 0.1, 1, P, None, P, big, None) == B.QLORA_ERR_MISALIGNED
+    assert fwd(P, 4, ctypes.byref(d), P, P, 16, 3e38, 0.5, 1, P, None, None, P, big, None) == B.QLORA_ERR_INVALID_ARG
+    assert fwd(P, 4, ctypes.byref(d), P, P, 16, 1.0, 0.1, 1, P, None, None, P, 1024, None) == B.QLORA_ERR_WORKSPACE
+    assert fwd(P + 2, 4, ctypes.byref(d), P, P, 16, 1.0, 0.1, 1, P, None, None, P, big, None) == B.QLORA_ERR_MISALIGNED
     bwd = lib.qlora_linear_bwd_dropout
-    assert bwd(P, P, 4, ctypes.byref(d), P, P, 16, 1.0, 1.0, 1, None, P, P, P, P, big, None) == B.QLORA_ERR_INVALID_ARG
-    assert bwd(P, P, 4, ctypes.byref(d), P, P, 16, 1.0, 0.1, 1, None, P, P, None, P, big, None) == B.QLORA_ERR_INVALID_ARG
-    assert bwd(P, P, 4, ctypes.byref(d), P, P, 16, 1.0, 0.1, 1, None, P, P, P, P, 8, None) == B.QLORA_ERR_WORKSPACE
+    assert bwd(P, P, 4, ctypes.byref(d), P, P, 16, 1.0, 1.0, 1, None, None, P, P, P, P, big, None) == B.QLORA_ERR_INVALID_ARG
+    assert bwd(P, P, 4, ctypes.byref(d), P, P, 16, 1.0, 0.1, 1, None, None, P, P, None, P, big, None) == B.QLORA_ERR_INVALID_ARG
+    assert bwd(P, P, 4, ctypes.byref(d), P, P, 16, 1.0, 0.1, 1, None, None, P, P, P, P, 8, None) == B.QLORA_ERR_WORKSPACE
+    # a mask buffer must be 16-byte aligned
+    assert fwd(P, 4, ctypes.byref(d), P, P, 16, 1.0, 0.1, 1, P, None, P + 4, P, big, None) == B.QLORA_ERR_MISALIGNED
+    assert bwd(P, P, 4, ctypes.byref(d), P, P, 16, 1.0, 0.1, 1, None, P + 4, P, P, P, P, big, None) == B.QLORA_ERR_MISALIGNED
     app = lib.qlora_dropout_apply
     assert app(None, 4, 128, 0.1, 1, P, None) == B.QLORA_ERR_INVALID_ARG
     assert app(P, 4, 128, 1.0, 1, P, None) == B.QLORA_ERR_INVALID_ARG

@@ -2,8 +2,9 @@
 LoRA dropout of 0.05 in the example configuration; read as inverted dropout on the adapter
 branch's input).
 
-The keep mask is checked bit for bit (qlora_dropout_apply against the oracle's own Philox4x32-10
-draw); the products within 2e-2 x RMS of the oracle's fp64 values for the same mask. Because
+The keep mask is checked bit for bit (qlora_dropout_apply and the forward's mask bits against the
+oracle's own Philox4x32-10 draw); the backward runs with the forward's mask and with a redrawn
+one; the products within 2e-2 x RMS of the oracle's fp64 values for the same mask. Because
 the adapter term is about 1% of Y and dX for the usual weight and adapter scales, a wrong mask
 there would hide under that bound: a zero weight (every code the zero level, scales 0, W' = 0
 exactly) leaves Y and dX with nothing but the adapter term, and dX must then be exactly 0 at
@@ -48,13 +49,17 @@ def test_dropout_mask_bit_exact(t, h, p, seed):
     assert np.array_equal(_bits(Xd), ref)
 
 
-def _run(li, p, seed, pass_sT=True):
+def _run(li, p, seed, pass_sT=True, pass_mask=True):
     P = B.nf4_quantize(li.Wt.cuda())
     X, L1, L2 = li.X.cuda(), li.L1.cuda(), li.L2.cuda()
-    Y, sT = B.qlora_linear_fwd_dropout(X, P, L1, L2, li.s, p, seed)
+    Y, sT, mask = B.qlora_linear_fwd_dropout(X, P, L1, L2, li.s, p, seed, want_mask=True)
     dX, dL1, dL2 = B.qlora_linear_bwd_dropout(li.dY.cuda(), X, P, L1, L2, li.s, p, seed,
-                                              sT=sT if pass_sT else None)
+                                              sT=sT if pass_sT else None,
+                                              mask=mask if pass_mask else None)
     assert B.last_status() == 0
+    keep = O.dropout_keep_mask(li.t, li.X.shape[1], p, seed)
+    assert np.array_equal(mask.cpu().numpy(), np.packbits(keep.reshape(-1), bitorder="little")), \
+        "mask bits"
     return P, Y, sT, dX, dL1, dL2
 
 
@@ -82,8 +87,8 @@ CASES = [
 def test_dropout_fwd_bwd(t, h, o, r, s, p, seed):
     li = inputs.random_linear(t, h, o, r, s, seed=700 + t + r)
     keep, *ref = _oracle(li, p, seed)
-    for pass_sT in (True, False):
-        _, *got = _run(li, p, seed, pass_sT)
+    for pass_sT, pass_mask in ((True, True), (False, False), (True, False)):
+        _, *got = _run(li, p, seed, pass_sT, pass_mask)
         for name, g, rf in zip(("Y", "sT", "dX", "dL1", "dL2"), got, ref):
             assert_close_rms(f32(g), rf, name)
 
@@ -107,7 +112,7 @@ def test_zero_weight_isolates_the_adapter_term(t, h, o, r, p):
     li.Wt.zero_()
     seed = 4000 + t
     keep, Y_ref, sT_ref, dX_ref, dL1_ref, dL2_ref = _oracle(li, p, seed)
-    _, Y, sT, dX, dL1, dL2 = _run(li, p, seed)
+    _, Y, sT, dX, dL1, dL2 = _run(li, p, seed, pass_mask=t % 2 == 0)
     for name, g, rf in (("sT", sT, sT_ref), ("dL1", dL1, dL1_ref), ("dL2", dL2, dL2_ref)):
         assert_close_rms(f32(g), rf, name)
     # Y and dX are nothing but the adapter term here, each through one bf16 intermediate
@@ -126,9 +131,10 @@ def test_p_zero_is_the_plain_layer_bit_for_bit():
     X, L1, L2, dY = li.X.cuda(), li.L1.cuda(), li.L2.cuda(), li.dY.cuda()
     Y0, sT0 = B.qlora_linear_fwd(X, P, L1, L2, li.s)
     g0 = B.qlora_linear_bwd(dY, X, P, L1, L2, li.s, sT=sT0)
-    Y1, sT1 = B.qlora_linear_fwd_dropout(X, P, L1, L2, li.s, 0.0, 77)
-    g1 = B.qlora_linear_bwd_dropout(dY, X, P, L1, L2, li.s, 0.0, 77, sT=sT1)
+    Y1, sT1, mask = B.qlora_linear_fwd_dropout(X, P, L1, L2, li.s, 0.0, 77, want_mask=True)
+    g1 = B.qlora_linear_bwd_dropout(dY, X, P, L1, L2, li.s, 0.0, 77, sT=sT1, mask=mask)
     assert B.last_status() == 0
+    assert bool((mask == 255).all())
     for a, b in zip((Y0, sT0, *g0), (Y1, sT1, *g1)):
         assert torch.equal(a, b)
 
