@@ -251,19 +251,6 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
           reinterpret_cast<uint4*>(args.out16b + off)[0] = o0;
           reinterpret_cast<uint4*>(args.out16b + off)[1] = o1;
         }
-      } else if (args.out_mode == kOutMaskBf16) {
-        // the element index row * Ncols + n0 is a multiple of 16 (n0 % 16 == 0, Ncols % 64 == 0)
-        const int64_t off = static_cast<int64_t>(row) * args.Ncols + n0;
-        const uint32_t keep = *reinterpret_cast<const uint16_t*>(args.keep_bits + off / 8);
-        const float a = args.alpha;
-        uint32_t o[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k)  // word k: element 2k in the low half, 2k + 1 high
-          o[k] = pack_bf16x2(((keep >> (2 * k)) & 1u) ? a * __uint_as_float(v[2 * k]) : 0.f,
-                             ((keep >> (2 * k + 1)) & 1u) ? a * __uint_as_float(v[2 * k + 1]) : 0.f);
-        uint4* d = reinterpret_cast<uint4*>(args.out16a + off);
-        d[0] = make_uint4(o[0], o[1], o[2], o[3]);
-        d[1] = make_uint4(o[4], o[5], o[6], o[7]);
       } else {
         float* dst = args.out32 + static_cast<int64_t>(row) * args.ld + n0;
 #pragma unroll
@@ -274,7 +261,52 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
       }
     };
     const int nchunks = BNp / 16;
-    if (ok && !*abort_flag && args.out_mode == kOutMergeNF4 && args.splits == 1) {
+    if (args.out_mode == kOutMaskBf16) {   // uniform over the block: all 128 threads reach
+                                           // the named barrier below
+      // The tile (128 rows x BNp bf16) is staged in the drained stage buffers, then written
+      // row by row by whole warps (512 contiguous bytes per warp store instead of 32 rows x 16
+      // bytes). Staging layout: 64-column blocks of 128 rows x 128 bytes, the 16-byte chunk
+      // index XORed with (row & 7), so that both the row-wise writes and the column-wise reads
+      // of eight consecutive threads hit eight distinct bank groups.
+      // After a timeout elsewhere in the CTA the tile is unspecified (the status word says so)
+      // but every access stays inside the stage buffers and the output.
+      uint8_t* stile = smem;
+      const bool go = __all_sync(0xFFFFFFFFu, ok && !*abort_flag);   // tcgen05.ld is warp-wide
+      const int rok = row < args.M;
+      const int64_t erow = static_cast<int64_t>(row) * args.Ncols;
+      for (int c = 0; go && c < nchunks; ++c) {
+        uint32_t v[16];
+        tmem_ld_16(lane_addr + c * 16, v);
+        tmem_ld_wait();
+        const int col = nb0 + c * 16;   // a multiple of 16: two bytes of mask bits
+        const uint32_t keep = (rok && col < args.Ncols)
+            ? *reinterpret_cast<const uint16_t*>(args.keep_bits + (erow + col) / 8) : 0u;
+        const float a = args.alpha;
+        uint32_t o[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)  // word k: element 2k in the low half, 2k + 1 high
+          o[k] = pack_bf16x2(((keep >> (2 * k)) & 1u) ? a * __uint_as_float(v[2 * k]) : 0.f,
+                             ((keep >> (2 * k + 1)) & 1u) ? a * __uint_as_float(v[2 * k + 1]) : 0.f);
+        const int blk = c >> 2, ch = (c & 3) * 2;   // 64-column block, first 16-byte chunk
+        uint8_t* rowp = stile + blk * (128 * 128) + rloc * 128;
+        *reinterpret_cast<uint4*>(rowp + (((ch) ^ (rloc & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(rowp + (((ch + 1) ^ (rloc & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");   // the four epilogue warps
+      const int chunks_row = BNp / 8;                     // 16-byte chunks per tile row
+      const int ncols_here = min(BNp, args.Ncols - nb0);
+      for (int rr = warp; go && rr < BM; rr += 4) {
+        const int grow = m0 + rr;
+        if (grow >= args.M) break;
+        for (int q = lane; q < chunks_row; q += 32) {
+          if (q * 8 >= ncols_here) break;
+          const int blk = q >> 3, ch = q & 7;
+          const uint4 val = *reinterpret_cast<const uint4*>(stile + blk * (128 * 128) + rr * 128 +
+                                                            ((ch ^ (rr & 7)) << 4));
+          *reinterpret_cast<uint4*>(args.out16a + static_cast<int64_t>(grow) * args.Ncols + nb0 + q * 8) = val;
+        }
+      }
+    } else if (ok && !*abort_flag && args.out_mode == kOutMergeNF4 && args.splits == 1) {
       // 64 columns (one NF4 block of this row) per round: the next block's 32 code bytes and
       // scales are loaded while this one's accumulator chunks come out of TMEM
       const int64_t rowbase = static_cast<int64_t>(row) * args.ld;
