@@ -330,6 +330,111 @@ def dequantize_bits_with(packed: NF4Packed, cb: int) -> np.ndarray:
     return bf16_bits_rne(nf4_dequantize_f32(packed, codebook_levels(cb)))
 
 
+# ----------------------------------------------------------------------------------------
+# Other 8-bit formats for the first-level scales ("QLoRA in LLMs" §1 "FP32, FP16, BF16, and
+# FP8": FP8 E4M3 has 4 exponent and 3 fraction bits, and FP8 and INT8 share one byte; §2 "Choose
+# a scale, then round": symmetric absmax to the integers -127 .. 127). The second level stays
+# one fp32 scale per 256 blocks; only the 8-bit code of each block scale changes:
+#   SCALES_U8   (the default) s2 = c2 / 255, q8 = clamp(rint(c1 / s2), 0, 255);
+#   SCALES_S8   the textbook signed scheme: s2 = c2 / 127, q8 = clamp(rint(c1 / s2), -127, 127)
+#               stored as the two's-complement byte (absmax scales are >= 0, so half the codes
+#               go unused: the point of the comparison);
+#   SCALES_E4M3 s2 = c2 / 448 (448 = the largest finite E4M3 value), q8 = the E4M3 code of
+#               c1 / s2 rounded to nearest even, saturating at 448.
+# E4M3 here is the 8-bit float with exponent bias 7, no infinities, and code 0x7F (and 0xFF)
+# as NaN, the variant tensor hardware converts to.
+# ----------------------------------------------------------------------------------------
+
+SCALES_U8, SCALES_S8, SCALES_E4M3 = 0, 1, 2
+E4M3_MAX = 448.0
+
+
+def e4m3_value(code) -> np.ndarray:
+    """Value of E4M3 codes (fp32): sign bit 7, exponent bits 6..3 (bias 7), fraction bits 2..0;
+    exponent 0 is subnormal (fraction x 2^-9); exponent 15 with fraction 7 is NaN."""
+    c = np.asarray(code, dtype=np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    v = sign * mag
+    v = np.where((e == 15) & (m == 7), np.nan, v)
+    return v.astype(np.float32)
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """E4M3 code (uint8) of non-negative finite fp32 values: the nearest finite E4M3 value, a tie
+    going to the even code (even fraction), values above 448 saturating to 448 (code 0x7E)."""
+    x = np.asarray(x, dtype=np.float64)
+    if np.any(~np.isfinite(x)) or np.any(x < 0):
+        raise ValueError("e4m3_encode takes non-negative finite values")
+    vals = e4m3_value(np.arange(0x7F)).astype(np.float64)   # codes 0x00 .. 0x7E, ascending
+    hi = np.clip(np.searchsorted(vals, x, side="left"), 0, 0x7E)
+    lo = np.clip(hi - 1, 0, 0x7E)
+    dlo, dhi = np.abs(x - vals[lo]), np.abs(vals[hi] - x)
+    pick = np.where(dlo < dhi, lo, np.where(dhi < dlo, hi, np.where(lo % 2 == 0, lo, hi)))
+    return pick.astype(np.uint8)
+
+
+def double_quantize_with(c1: np.ndarray, fmt: int):
+    """Second-level quantization of the block scales in scale format `fmt` (see above);
+    groups of 256 blocks as in double_quantize."""
+    if fmt == SCALES_U8:
+        return double_quantize(c1)
+    c1 = np.asarray(c1, dtype=np.float32)
+    nb = c1.size
+    ng = (nb + GROUP - 1) // GROUP
+    q8 = np.zeros(nb, dtype=np.uint8)
+    s2 = np.zeros(ng, dtype=np.float32)
+    for g in range(ng):
+        seg = c1[g * GROUP:(g + 1) * GROUP]
+        if fmt == SCALES_S8:
+            codes, scale = absmax_int_quantize(seg, 127, signed=True)
+            q8[g * GROUP:(g + 1) * GROUP] = codes.astype(np.int8).view(np.uint8)
+            s2[g] = scale
+        elif fmt == SCALES_E4M3:
+            c2 = np.float32(np.max(seg))
+            scale = np.float32(c2 / np.float32(E4M3_MAX))
+            s2[g] = scale
+            if scale == 0.0:
+                continue
+            q8[g * GROUP:(g + 1) * GROUP] = e4m3_encode((seg / scale).astype(np.float32))
+        else:
+            raise ValueError("unknown scale format")
+    return q8, s2
+
+
+def scale_code_values(q8: np.ndarray, fmt: int) -> np.ndarray:
+    """The number each 8-bit scale code stands for (fp32, exact)."""
+    q8 = np.asarray(q8, dtype=np.uint8)
+    if fmt == SCALES_U8:
+        return q8.astype(np.float32)
+    if fmt == SCALES_S8:
+        return q8.view(np.int8).astype(np.float32)
+    if fmt == SCALES_E4M3:
+        return e4m3_value(q8)
+    raise ValueError("unknown scale format")
+
+
+def quantize_format(Wt: np.ndarray, cb: int, fmt: int) -> NF4Packed:
+    """quantize_with(Wt, cb) with the block scales in scale format `fmt`; the 4-bit codes do
+    not depend on the scale format (they use the exact c1)."""
+    p = quantize_with(Wt, cb)
+    p.absmax_q8, p.absmax_s2 = double_quantize_with(p.absmax_f32, fmt)
+    return p
+
+
+def dequantize_bits_format(packed: NF4Packed, cb: int, fmt: int) -> np.ndarray:
+    """bf16 bit patterns of bf16(level[code] * (value(q8) * s2)), two fp32 multiplies."""
+    q = codebook_levels(cb)
+    codes = unpack_nibbles(packed.codes).reshape(-1, BLOCK)
+    g = np.arange(packed.absmax_q8.size) // GROUP
+    k = (scale_code_values(packed.absmax_q8, fmt) *
+         np.asarray(packed.absmax_s2, dtype=np.float32)[g]).astype(np.float32)
+    w = (q[codes] * k[:, None]).astype(np.float32)
+    return bf16_bits_rne(w.reshape(packed.out_features, packed.in_features))
+
+
 def block_scales(q8: np.ndarray, s2: np.ndarray) -> np.ndarray:
     """Reconstructed first-level scale per block: float(q8[b]) * s2[b // 256] (fp32)."""
     q8 = np.asarray(q8, dtype=np.uint8)
