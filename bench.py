@@ -401,24 +401,29 @@ def stack65b_leg(dev, peaks, steps: int = 2, warmup: int = 1):
 def codebook_leg(dev):
     """The pages' format comparison on the LLaMA-7B-shaped layer's weights: relative
     reconstruction error (sum of squared errors / sum of squares) of NF4, FP4 and INT4 packing
-    (same blocks and double-quantized scales), on N(0, 0.02) weights with the 1% outliers at
-    8 sigma of the quantization workload and without them, and the quantizer's time for each."""
+    (same blocks and double-quantized scales), and of NF4 with the block scales in signed int8
+    (/127) and FP8 E4M3 instead of unsigned 8-bit, on N(0, 0.02) weights with the 1% outliers
+    at 8 sigma of the quantization workload and without them, and the quantizer's time for each."""
     from bit_quantized_lora_03_b200 import binding as B
     from bit_quantized_lora_03_b200 import inputs
     res = {}
+    variants = (("nf4", B.CODEBOOK_NF4, B.SCALES_U8), ("fp4", B.CODEBOOK_FP4, B.SCALES_U8),
+                ("int4", B.CODEBOOK_INT4, B.SCALES_U8),
+                ("nf4_scales_s8", B.CODEBOOK_NF4, B.SCALES_S8),
+                ("nf4_scales_e4m3", B.CODEBOOK_NF4, B.SCALES_E4M3))
     for tag, outl in (("with_outliers", True), ("gaussian", False)):
         W = [w.to(dev) for _, w in inputs.llama7b_quant_weights(with_outliers=outl)]
         res[tag] = {}
-        for name, cb in (("nf4", B.CODEBOOK_NF4), ("fp4", B.CODEBOOK_FP4), ("int4", B.CODEBOOK_INT4)):
+        for name, cb, fmt in variants:
             packs = [B.PackedNF4(w.shape[0], w.shape[1], dev) for w in W]
 
             def quant():
                 for w, p in zip(W, packs):
-                    B.nf4_quantize(w, out=p, codebook_id=cb)
+                    B.nf4_quantize(w, out=p, codebook_id=cb, scale_format=fmt)
             ms = queued_ms(quant, 3, 1) / 3
             se, ss = 0.0, 0.0
             for w, p in zip(W, packs):
-                d = B.nf4_dequantize(p, codebook_id=cb).float()
+                d = B.nf4_dequantize(p, codebook_id=cb, scale_format=fmt).float()
                 se += float((d - w).pow(2).sum())
                 ss += float(w.pow(2).sum())
             res[tag][name] = {"rel_mse": round(se / ss, 6), "quantize_ms": round(ms, 4)}
@@ -686,6 +691,8 @@ def main():
                     help="profiling case: only linear I of the layer, fwd+bwd, no extras")
     ap.add_argument("--dropout", type=float, default=0.0, metavar="P",
                     help="with --single-linear: LoRA dropout P on the adapter input")
+    ap.add_argument("--codebooks-only", action="store_true",
+                    help="run only the codebook / scale-format comparison leg and print it")
     ap.add_argument("--dropout-only", action="store_true",
                     help="after the headline, run only the LoRA-dropout leg (no other legs, no CPU baseline)")
     ap.add_argument("--decode-case", type=int, nargs=2, default=None, metavar=("T", "I"),
@@ -714,6 +721,9 @@ def main():
 
     if args.decode_case is not None:
         return decode_case(B, dev, *args.decode_case)
+    if args.codebooks_only:
+        print(json.dumps(codebook_leg(dev)), flush=True)
+        return 0
     t, r, s = args.tokens, 64, 0.25
     if args.single_linear is not None:
         L = Layer(args.single_linear, dev, t, r, s)

@@ -53,6 +53,8 @@ SIGNATURES = {
                                         ctypes.c_float, _I64, ctypes.c_uint, _PTR]),
     "qlora_quantize_codebook": (ctypes.c_int, [_PTR, _PTR, ctypes.c_int, _PTR]),
     "qlora_dequantize_codebook": (ctypes.c_int, [_PTR, ctypes.c_int, _PTR, _PTR]),
+    "qlora_quantize_format": (ctypes.c_int, [_PTR, _PTR, ctypes.c_int, ctypes.c_int, _PTR]),
+    "qlora_dequantize_format": (ctypes.c_int, [_PTR, ctypes.c_int, ctypes.c_int, _PTR, _PTR]),
     "qlora_profile_begin": (ctypes.c_int, [ctypes.c_int]),
     "qlora_profile_end": (ctypes.c_int, [_PTR, _PTR, ctypes.c_int]),
     "qlora_kernel_name": (ctypes.c_char_p, [ctypes.c_int]),
@@ -124,6 +126,7 @@ def _ptr(t: torch.Tensor | None) -> int | None:
 
 
 CODEBOOK_NF4, CODEBOOK_FP4, CODEBOOK_INT4 = 0, 1, 2
+SCALES_U8, SCALES_S8, SCALES_E4M3 = 0, 1, 2
 
 
 def codebook(codebook_id: int | None = None):
@@ -168,14 +171,18 @@ def _require(t: torch.Tensor, dtype, shape, name: str) -> None:
 
 
 def nf4_quantize(Wt: torch.Tensor, out: PackedNF4 | None = None, stream=None,
-                 codebook_id: int = CODEBOOK_NF4) -> PackedNF4:
+                 codebook_id: int = CODEBOOK_NF4, scale_format: int = SCALES_U8) -> PackedNF4:
     """Quantize an fp32 CUDA weight Wt (o x h) to packed 4-bit codes with double-quantized
-    scales (NF4 unless another codebook id is given)."""
+    scales (NF4 and unsigned 8-bit scales unless another codebook or scale format is given)."""
     o, h = Wt.shape
     _require(Wt, torch.float32, (o, h), "Wt")
     p = out if out is not None else PackedNF4(o, h, Wt.device)
     d = p.desc()
-    if codebook_id == CODEBOOK_NF4:
+    if scale_format != SCALES_U8:
+        _check(lib().qlora_quantize_format(Wt.data_ptr(), ctypes.byref(d), int(codebook_id),
+                                           int(scale_format), _stream(stream)),
+               "qlora_quantize_format")
+    elif codebook_id == CODEBOOK_NF4:
         _check(lib().nf4_quantize(Wt.data_ptr(), ctypes.byref(d), _stream(stream)), "nf4_quantize")
     else:
         _check(lib().qlora_quantize_codebook(Wt.data_ptr(), ctypes.byref(d), int(codebook_id),
@@ -184,15 +191,19 @@ def nf4_quantize(Wt: torch.Tensor, out: PackedNF4 | None = None, stream=None,
 
 
 def nf4_dequantize(p: PackedNF4, out: torch.Tensor | None = None, stream=None,
-                   codebook_id: int = CODEBOOK_NF4) -> torch.Tensor:
-    """The bf16 weight Wt' (o x h) reconstructed from a packed weight (with the codebook it
-    was packed with)."""
+                   codebook_id: int = CODEBOOK_NF4, scale_format: int = SCALES_U8) -> torch.Tensor:
+    """The bf16 weight Wt' (o x h) reconstructed from a packed weight (with the codebook and
+    scale format it was packed with)."""
     if out is None:
         out = torch.empty(p.out_features, p.in_features, dtype=torch.bfloat16,
                           device=p.codes.device)
     _require(out, torch.bfloat16, (p.out_features, p.in_features), "out")
     d = p.desc()
-    if codebook_id == CODEBOOK_NF4:
+    if scale_format != SCALES_U8:
+        _check(lib().qlora_dequantize_format(ctypes.byref(d), int(codebook_id), int(scale_format),
+                                             out.data_ptr(), _stream(stream)),
+               "qlora_dequantize_format")
+    elif codebook_id == CODEBOOK_NF4:
         _check(lib().nf4_dequantize(ctypes.byref(d), out.data_ptr(), _stream(stream)),
                "nf4_dequantize")
     else:

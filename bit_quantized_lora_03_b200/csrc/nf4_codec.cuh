@@ -9,6 +9,8 @@
 // IEEE round-to-nearest ones the method's definition fixes (__fdiv_rn, __fmul_rn, rint).
 #pragma once
 
+#include <cuda_fp8.h>
+
 #include "qlora_common.cuh"
 
 namespace qlora {
@@ -83,6 +85,37 @@ __device__ __forceinline__ float fmax_nan(float a, float b) {
 // into one of two 64 KB shared-memory buffers with bulk copies, one group ahead, so HBM reads
 // overlap the previous group's arithmetic. Half-warp h of pass p (0..7) owns block 32p + h;
 // each of its lanes reads one float4 of the block from shared memory.
+// 8-bit formats of the block scales ("QLoRA in LLMs" section 1: FP8 E4M3 has 4 exponent and 3
+// fraction bits; section 2 "Choose a scale, then round": symmetric absmax to -127 .. 127). The
+// second level is one fp32 scale s2 per 256 blocks in every format:
+//   kScalesU8   s2 = c2 / 255, q8 = clamp(rint(c1 / s2), 0, 255)             (the default)
+//   kScalesS8   s2 = c2 / 127, q8 = clamp(rint(c1 / s2), -127, 127) as a two's-complement byte
+//   kScalesE4M3 s2 = c2 / 448, q8 = E4M3 code of c1 / s2 (round to nearest even, saturating)
+enum ScaleFormat : int { kScalesU8 = 0, kScalesS8 = 1, kScalesE4M3 = 2 };
+
+__host__ __device__ constexpr float scale_format_top(int sfmt) {
+  return sfmt == kScalesU8 ? 255.0f : (sfmt == kScalesS8 ? 127.0f : 448.0f);
+}
+
+__device__ __forceinline__ uint8_t scale_code(float c1, float s2, int sfmt) {
+  if (s2 == 0.0f) return 0;
+  const float x = __fdiv_rn(c1, s2);
+  if (sfmt == kScalesE4M3)
+    return static_cast<uint8_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3));
+  const int lo = sfmt == kScalesS8 ? -127 : 0, hi = sfmt == kScalesS8 ? 127 : 255;
+  return static_cast<uint8_t>(min(hi, max(lo, __float2int_rn(x))));
+}
+
+// The number an 8-bit scale code stands for (exact in fp32).
+__device__ __forceinline__ float scale_code_value(uint8_t q, int sfmt) {
+  if (sfmt == kScalesS8) return static_cast<float>(static_cast<int8_t>(q));
+  if (sfmt == kScalesE4M3) {
+    const __half_raw hr = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(q), __NV_E4M3);
+    return __half2float(__half(hr));
+  }
+  return static_cast<float>(q);
+}
+
 namespace qz {
 constexpr int kThreads = 512;
 constexpr int kGroupBytes = kGroup * kBlock * 4;  // 64 KB
@@ -92,7 +125,7 @@ constexpr size_t smem_bytes() { return 2 * static_cast<size_t>(kGroupBytes) + 64
 
 __global__ void __launch_bounds__(qz::kThreads, 1) nf4_quantize_kernel(
     const float* __restrict__ W, uint8_t* __restrict__ codes, uint8_t* __restrict__ q8,
-    float* __restrict__ s2, int64_t nblocks, Nf4Table tab, Nf4Buckets bkt) {
+    float* __restrict__ s2, int64_t nblocks, Nf4Table tab, Nf4Buckets bkt, int sfmt) {
   extern __shared__ __align__(128) uint8_t qsm[];
   __shared__ float mids[16];
   __shared__ __align__(16) float2 bk[128 * 32];  // [bucket][lane]
@@ -178,7 +211,7 @@ __global__ void __launch_bounds__(qz::kThreads, 1) nf4_quantize_kernel(
       fence_proxy_async_smem();  // the reads above come before the copy that overwrites b
       issue(g + 2 * static_cast<int64_t>(gridDim.x), b);
     }
-    // second level: c2 = max over the group's block scales; s2 = c2 / 255; q8 = rint(c1 / s2)
+    // second level: c2 = max over the group's block scales; s2 = c2 / top; q8 = code(c1 / s2)
     const float c1 = (tid < nb) ? c1s[tid] : 0.0f;
     float m = c1;
 #pragma unroll
@@ -188,12 +221,8 @@ __global__ void __launch_bounds__(qz::kThreads, 1) nf4_quantize_kernel(
     float c2 = wmax[0];
 #pragma unroll
     for (int i = 1; i < qz::kThreads / 32; ++i) c2 = fmaxf(c2, wmax[i]);
-    const float sc = __fdiv_rn(c2, 255.0f);
-    if (tid < nb) {
-      int qv = 0;
-      if (sc != 0.0f) qv = min(255, max(0, __float2int_rn(__fdiv_rn(c1, sc))));
-      q8[g * kGroup + tid] = static_cast<uint8_t>(qv);
-    }
+    const float sc = __fdiv_rn(c2, scale_format_top(sfmt));
+    if (tid < nb) q8[g * kGroup + tid] = scale_code(c1, sc, sfmt);
     if (tid == 0) s2[g] = sc;
     __syncthreads();  // c1s and wmax are rewritten by the next group
   }
@@ -207,7 +236,8 @@ __global__ void __launch_bounds__(256) nf4_dequantize_kernel(const uint8_t* __re
                                                              const uint8_t* __restrict__ q8,
                                                              const float* __restrict__ s2,
                                                              uint16_t* __restrict__ out,
-                                                             int64_t nitems, Nf4Table tab) {
+                                                             int64_t nitems, Nf4Table tab,
+                                                             int sfmt) {
   __shared__ float lv[16];
   if (threadIdx.x < 16) lv[threadIdx.x] = tab.level[threadIdx.x];
   __syncthreads();
@@ -222,7 +252,7 @@ __global__ void __launch_bounds__(256) nf4_dequantize_kernel(const uint8_t* __re
       if (it < nitems) {
         w[u] = __ldcs(reinterpret_cast<const unsigned int*>(codes) + it);
         const int64_t b = it >> 3;  // 8 items per 64-weight block
-        k[u] = __fmul_rn(static_cast<float>(__ldg(q8 + b)), __ldg(s2 + (b >> 8)));
+        k[u] = __fmul_rn(scale_code_value(__ldg(q8 + b), sfmt), __ldg(s2 + (b >> 8)));
       }
     }
 #pragma unroll

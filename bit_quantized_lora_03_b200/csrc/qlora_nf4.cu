@@ -1001,10 +1001,11 @@ int qlora_get_last_status(qlora_stream_t stream) {
   return static_cast<int>(v);
 }
 
-int qlora_quantize_codebook(const float* Wt, const nf4_weight* q, int codebook_id,
-                            qlora_stream_t stream) {
+int qlora_quantize_format(const float* Wt, const nf4_weight* q, int codebook_id, int scale_format,
+                          qlora_stream_t stream) {
   if (!Wt) return QLORA_ERR_INVALID_ARG;
   if (codebook_id < 0 || codebook_id >= kCodebooks) return QLORA_ERR_INVALID_ARG;
+  if (scale_format < kScalesU8 || scale_format > kScalesE4M3) return QLORA_ERR_INVALID_ARG;
   int rc = check_weight(q);
   if (rc) return rc;
   if (!aligned16(Wt)) return QLORA_ERR_MISALIGNED;
@@ -1017,15 +1018,16 @@ int qlora_quantize_codebook(const float* Wt, const nf4_weight* q, int codebook_i
     prof::Scope ps(prof::kQuant, reinterpret_cast<cudaStream_t>(stream));
     nf4_quantize_kernel<<<grid, qz::kThreads, qz::smem_bytes(), reinterpret_cast<cudaStream_t>(stream)>>>(
         Wt, q->codes, q->absmax_q8, q->absmax_s2, nblocks, device_table(codebook_id),
-        device_buckets(codebook_id));
+        device_buckets(codebook_id), scale_format);
   }
   return launch_status();
 }
 
-int qlora_dequantize_codebook(const nf4_weight* q, int codebook_id, uint16_t* Wt_out,
-                              qlora_stream_t stream) {
+int qlora_dequantize_format(const nf4_weight* q, int codebook_id, int scale_format, uint16_t* Wt_out,
+                            qlora_stream_t stream) {
   if (!Wt_out) return QLORA_ERR_INVALID_ARG;
   if (codebook_id < 0 || codebook_id >= kCodebooks) return QLORA_ERR_INVALID_ARG;
+  if (scale_format < kScalesU8 || scale_format > kScalesE4M3) return QLORA_ERR_INVALID_ARG;
   int rc = check_weight(q);
   if (rc) return rc;
   if (!aligned16(Wt_out)) return QLORA_ERR_MISALIGNED;
@@ -1037,9 +1039,20 @@ int qlora_dequantize_codebook(const nf4_weight* q, int codebook_id, uint16_t* Wt
   {
     prof::Scope ps(prof::kDequant, reinterpret_cast<cudaStream_t>(stream));
     nf4_dequantize_kernel<<<std::max(grid, 1), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        q->codes, q->absmax_q8, q->absmax_s2, Wt_out, nitems, device_table(codebook_id));
+        q->codes, q->absmax_q8, q->absmax_s2, Wt_out, nitems, device_table(codebook_id),
+        scale_format);
   }
   return launch_status();
+}
+
+int qlora_quantize_codebook(const float* Wt, const nf4_weight* q, int codebook_id,
+                            qlora_stream_t stream) {
+  return qlora_quantize_format(Wt, q, codebook_id, kScalesU8, stream);
+}
+
+int qlora_dequantize_codebook(const nf4_weight* q, int codebook_id, uint16_t* Wt_out,
+                              qlora_stream_t stream) {
+  return qlora_dequantize_format(q, codebook_id, kScalesU8, Wt_out, stream);
 }
 
 int nf4_quantize(const float* Wt, const nf4_weight* q, qlora_stream_t stream) {

@@ -266,6 +266,29 @@ QLORA_API int qlora_quantize_codebook(const float *Wt, const nf4_weight *q, int 
 QLORA_API int qlora_dequantize_codebook(const nf4_weight *q, int codebook_id, uint16_t *Wt_out,
                                         qlora_stream_t stream);
 
+/* Other 8-bit formats for the double-quantized block scales ("QLoRA in LLMs" section 1, "FP32,
+ * FP16, BF16, and FP8": E4M3 has 4 exponent and 3 fraction bits; section 2, "Choose a scale,
+ * then round": symmetric absmax to the integers -127 .. 127). The second level is one fp32
+ * scale s2 per 256 blocks in every format; c1 is a block's absmax, c2 its group's largest c1:
+ *   QLORA_SCALES_U8 (0)    s2 = c2 / 255, q8 = clamp(rint(c1 / s2), 0, 255)  (nf4_quantize's)
+ *   QLORA_SCALES_S8 (1)    s2 = c2 / 127, q8 = clamp(rint(c1 / s2), -127, 127), stored as the
+ *                          two's-complement byte (the textbook signed scheme; codes < 0 unused)
+ *   QLORA_SCALES_E4M3 (2)  s2 = c2 / 448, q8 = the FP8 E4M3 code (bias 7, no infinities, 0x7F
+ *                          NaN) of c1 / s2 rounded to nearest even, saturating at 448
+ * Dequantization: w' = bf16_rn(level[code] * (value(q8) * s2)). The 4-bit codes do not depend
+ * on the scale format. A weight must be dequantized with the codebook and scale format it was
+ * packed with; only NF4 with QLORA_SCALES_U8 may be passed to the linear calls. The
+ * _codebook calls are these with QLORA_SCALES_U8.
+ * Errors: QLORA_ERR_INVALID_ARG for an unknown id or format, else as nf4_quantize /
+ * nf4_dequantize. */
+#define QLORA_SCALES_U8 0
+#define QLORA_SCALES_S8 1
+#define QLORA_SCALES_E4M3 2
+QLORA_API int qlora_quantize_format(const float *Wt, const nf4_weight *q, int codebook_id,
+                                    int scale_format, qlora_stream_t stream);
+QLORA_API int qlora_dequantize_format(const nf4_weight *q, int codebook_id, int scale_format,
+                                      uint16_t *Wt_out, qlora_stream_t stream);
+
 /* Adapter merge ("QLoRA in LLMs" section 11, "Saving, Loading, and Merging QLoRA Adapters":
  * dequantize the base into a wider precision, add the LoRA update, optionally quantize the
  * result again): Wt_merged = W'^T + s . (L1 . L2)^T, i.e. W_m = W' + s.L1.L2 in the stored

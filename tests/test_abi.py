@@ -126,6 +126,21 @@ def test_unknown_codebook_is_rejected(lib):
     assert lib.qlora_codebook(-1, ctypes.cast(lv, ctypes.c_void_p), None) == B.QLORA_ERR_INVALID_ARG
 
 
+def test_scale_format_argument_checks(lib):
+    d = _desc()
+    q = ctypes.byref(d)
+    P = 0x10000
+    for fmt in (-1, 3, 99):
+        assert lib.qlora_quantize_format(P, q, 0, fmt, None) == B.QLORA_ERR_INVALID_ARG
+        assert lib.qlora_dequantize_format(q, 0, fmt, P, None) == B.QLORA_ERR_INVALID_ARG
+    assert lib.qlora_quantize_format(P, q, 3, B.SCALES_S8, None) == B.QLORA_ERR_INVALID_ARG
+    assert lib.qlora_quantize_format(None, q, 0, B.SCALES_E4M3, None) == B.QLORA_ERR_INVALID_ARG
+    assert lib.qlora_quantize_format(P + 4, q, 0, B.SCALES_E4M3, None) == B.QLORA_ERR_MISALIGNED
+    assert lib.qlora_dequantize_format(q, 0, B.SCALES_S8, P + 2, None) == B.QLORA_ERR_MISALIGNED
+    bad_h = _desc(h=100)
+    assert lib.qlora_dequantize_format(ctypes.byref(bad_h), 0, B.SCALES_S8, P, None) == B.QLORA_ERR_BAD_SHAPE
+
+
 def test_adamw_argument_checks(lib):
     f = lib.qlora_adamw_step
     p = ctypes.c_void_p(16)   # never dereferenced: the checks run before anything else

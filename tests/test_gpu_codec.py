@@ -136,3 +136,31 @@ def test_other_codebooks_bit_exact(cb):
     W[3] = 0.0
     W[10, :64] = 0.0
     _check_codebook(W, cb)
+
+
+def _check_format(Wt: torch.Tensor, cb: int, fmt: int):
+    p = B.nf4_quantize(Wt.cuda(), codebook_id=cb, scale_format=fmt)
+    deq = B.nf4_dequantize(p, codebook_id=cb, scale_format=fmt)
+    assert B.last_status() == 0
+    ref = O.quantize_format(Wt.numpy(), cb, fmt)
+    assert np.array_equal(p.codes.cpu().numpy(), ref.codes)
+    assert np.array_equal(p.absmax_q8.cpu().numpy(), ref.absmax_q8)
+    assert np.array_equal(p.absmax_s2.cpu().numpy().view(np.uint32), ref.absmax_s2.view(np.uint32))
+    assert np.array_equal(deq.view(torch.int16).cpu().numpy().view(np.uint16),
+                          O.dequantize_bits_format(ref, cb, fmt))
+
+
+@pytest.mark.parametrize("fmt", [B.SCALES_S8, B.SCALES_E4M3])
+@pytest.mark.parametrize("cb", [B.CODEBOOK_NF4, B.CODEBOOK_FP4])
+def test_other_scale_formats_bit_exact(cb, fmt):
+    """Signed int8 and FP8 E4M3 block scales, bit for bit: a LLaMA-7B q_proj with 1% outliers
+    (scales spread over the whole code range, E4M3 subnormals among them), a ragged shape with
+    all-zero blocks and a group whose scales are all zero, and blocks of tiny magnitude."""
+    _check_format(inputs.weight_f32(4096, 4096, 200, outliers=True), cb, fmt)
+    g = torch.Generator().manual_seed(10 + fmt)
+    W = torch.randn(257, 192, generator=g) * 0.02
+    W[3] = 0.0
+    W[10, :64] = 0.0
+    W[20:40] *= 1e-5          # block scales far below the group's largest: E4M3 subnormals
+    W[160:] = 0.0             # blocks 480 .. 770 zero: second-level group 2 entirely zero
+    _check_format(W, cb, fmt)
