@@ -1,8 +1,10 @@
 // Plain TMA-fed tcgen05 GEMM for the rank-r products of the QLoRA linear on sm_100a:
 // T = X.L1 and U = dY.L2^T (rounded to bf16 sT, sU) and the adapter gradients dL1 = X^T.sU and
-// dL2^T = dY^T.sT ("The algebra", mchromiak.github.io; "QLoRA in LLMs" sections 3-4). Both
-// operands by TMA (either major-ness), one N tile (N <= 256), split-K as one thread-block
-// cluster whose CTAs reduce through distributed shared memory.
+// dL2^T = dY^T.sT ("The algebra", mchromiak.github.io; "QLoRA in LLMs" sections 3-4); with
+// epilogue variants for the adapter merge (W' + s.L1.L2, "QLoRA in LLMs" section 11) and the
+// dropout-masked adapter term of dX (section 12). Both operands by TMA (either major-ness),
+// N tiles of up to 256 columns, split-K as one thread-block cluster whose CTAs reduce through
+// distributed shared memory.
 //
 // Every wait is bounded (qlora::mbar_wait); on expiry the CTA reports QLORA_DEV_TIMEOUT,
 // stops issuing, waits for its own copies and MMAs in flight, frees TMEM and returns.
