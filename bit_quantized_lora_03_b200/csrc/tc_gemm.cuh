@@ -394,13 +394,22 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
     const int tile_cols = args.Ncols - nb0 < BNp ? args.Ncols - nb0 : BNp;
     if (!*abort_flag) {
       if (args.out_mode == kOutTransposed) {
-        // consecutive threads take consecutive rows of one column: coalesced column stores
-        for (int e = threadIdx.x; e < nr * tile_cols; e += kThreads) {
-          const int rl = r0 + e % nr, n = e / nr;
-          float sum = 0.f;
-          for (int p = 0; p < S; ++p) sum += ld_dsmem_f32(part0 + rl * ld_s + n, static_cast<uint32_t>(p));
-          if (m0 + rl < args.M && nb0 + n < args.Ncols)
-            args.out32[static_cast<int64_t>(nb0 + n) * args.ld + m0 + rl] = sum;
+        // four adjacent columns per thread (one 16-byte read from each rank); consecutive
+        // threads take consecutive rows, so each of the four column stores is coalesced
+        const int nq = tile_cols / 4;
+        for (int e = threadIdx.x; e < nr * nq; e += kThreads) {
+          const int rl = r0 + e % nr, n = 4 * (e / nr);
+          float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int p = 0; p < S; ++p) {
+            const float4 v = ld_dsmem_f32x4(part0 + rl * ld_s + n, static_cast<uint32_t>(p));
+            sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+          }
+          if (m0 + rl >= args.M || nb0 + n >= args.Ncols) continue;
+          float* o = args.out32 + static_cast<int64_t>(nb0 + n) * args.ld + m0 + rl;
+          o[0] = sum.x;
+          o[args.ld] = sum.y;
+          o[2 * args.ld] = sum.z;
+          o[3 * args.ld] = sum.w;
         }
       } else {
         const int nq = tile_cols / 4;
