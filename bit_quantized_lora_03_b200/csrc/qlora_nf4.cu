@@ -388,6 +388,17 @@ TcPlan plan_tc(int64_t M, int64_t ncols, int64_t K, bool b_mn, int sms) {
   int splits = std::max(1, sms / p.mtiles);
   splits = std::min(splits, std::max(1, p.num_kb / 4));
   splits = std::min(splits, kMaxTcSplits);  // split-K is one cluster (portable size)
+  // Between sms/2 and sms row tiles (e.g. 86 for an 11008-row output) one CTA per tile leaves
+  // SMs idle: split K in two and halve the pipeline so that two CTAs fit on an SM.
+  if (splits == 1 && p.mtiles < sms && p.num_kb >= 8) {
+    int st2 = stages;
+    while (st2 > 2 && 2 * tcg::smem_bytes(st2, p.BNp, b_mn) > static_cast<size_t>(tcg::kSmemPerSm)) --st2;
+    if (2 * tcg::smem_bytes(st2, p.BNp, b_mn) <= static_cast<size_t>(tcg::kSmemPerSm)) {
+      splits = 2;
+      p.stages = st2;
+      p.smem = tcg::smem_bytes(st2, p.BNp, b_mn);
+    }
+  }
 #ifdef QLORA_TUNING
   if (const char* e = std::getenv("QLORA_TC_WAVE")) splits = std::max(1, (std::atoi(e) * sms) / p.mtiles);
   if (const char* e = std::getenv("QLORA_TC_MINKB")) splits = std::min(splits, std::max(1, p.num_kb / std::atoi(e)));

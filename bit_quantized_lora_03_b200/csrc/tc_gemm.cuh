@@ -26,6 +26,7 @@ constexpr int A_BYTES = BM * BK * 2;        // 16 KB
 constexpr int kThreads = 6 * 32;            // warps 0-3 epilogue, 4 TMA, 5 MMA
 constexpr int kTmaWarp = 4, kMmaWarp = 5;
 constexpr int kMaxSmem = 232448 - 1024;     // opt-in maximum per CTA on sm_100, less static smem
+constexpr int kSmemPerSm = 233472 - 4096;   // shared memory of one SM, less two CTAs' reserve and static arrays
 // B tile bytes for a given MMA N (BNp, multiple of 16) and major-ness
 __host__ __device__ constexpr int b_bytes(int BNp, bool b_mn) {
   return b_mn ? ((BNp + 63) / 64) * 8192 : BNp * 128;
