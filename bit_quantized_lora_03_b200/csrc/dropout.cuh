@@ -74,9 +74,9 @@ __device__ __forceinline__ uint32_t keep_halves(uint32_t keep, int k2) {
 // generator call), so that enough bytes are in flight to cover the memory latency.
 constexpr int kDropUnroll = 4;
 
+// X and Xd may be the same buffer: each 16-byte group is read and written by one thread.
 template <bool kFromBits>
-__global__ void __launch_bounds__(256) dropout_apply_kernel(const uint4* __restrict__ X,
-                                                            uint4* __restrict__ Xd,
+__global__ void __launch_bounds__(256) dropout_apply_kernel(const uint4* X, uint4* Xd,
                                                             uint8_t* __restrict__ bits,
                                                             int64_t n8, DropoutKey key) {
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;

@@ -1119,6 +1119,9 @@ int qlora_dropout_apply(const uint16_t* X, int64_t t, int64_t h, float p, uint64
   if (!X || !Xd || !valid_dropout_p(p)) return QLORA_ERR_INVALID_ARG;
   if (t < 1 || h < 64 || h % 64 != 0 || t >= kMaxDim || h >= kMaxDim) return QLORA_ERR_BAD_SHAPE;
   if (!aligned16(X) || !aligned16(Xd)) return QLORA_ERR_MISALIGNED;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(X), b = reinterpret_cast<uintptr_t>(Xd);
+  const uintptr_t bytes = static_cast<uintptr_t>(t) * static_cast<uintptr_t>(h) * 2u;
+  if (a != b && a < b + bytes && b < a + bytes) return QLORA_ERR_INVALID_ARG;  // partial overlap
   int dev, rc;
   if ((rc = current_device(&dev))) return rc;
   return launch_dropout_apply(X, t * h, Xd, nullptr, false, dropout_key(p, seed), sm_count(dev),

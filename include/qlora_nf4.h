@@ -221,8 +221,9 @@ QLORA_API size_t qlora_bwd_dropout_workspace_bytes(int64_t t, int64_t h, int64_t
 
 /* qlora_dropout_apply -- Xd = X (.) M for the mask above (dropped elements become +0; no
  * 1 / (1 - p) scaling), so that the mask can be inspected on its own.
- *   X, Xd  device bf16, t x h row-major (may not overlap unless equal).  h % 64 == 0.
- * Errors: INVALID_ARG (NULL, p outside [0, 1)), BAD_SHAPE, MISALIGNED. */
+ *   X, Xd  device bf16, t x h row-major; Xd == X works in place, any other overlap is
+ *          rejected.  h % 64 == 0.
+ * Errors: INVALID_ARG (NULL, p outside [0, 1), partial overlap), BAD_SHAPE, MISALIGNED. */
 QLORA_API int qlora_dropout_apply(const uint16_t *X, int64_t t, int64_t h, float p, uint64_t seed,
                                   uint16_t *Xd, qlora_stream_t stream);
 

@@ -191,5 +191,6 @@ def test_dropout_workspace_and_argument_checks(lib):
     assert app(P, 4, 100, 0.1, 1, P, None) == B.QLORA_ERR_BAD_SHAPE
     assert app(P, 0, 128, 0.1, 1, P, None) == B.QLORA_ERR_BAD_SHAPE
     assert app(P, 4, 128, 0.1, 1, P + 8, None) == B.QLORA_ERR_MISALIGNED
+    assert app(P, 4, 128, 0.1, 1, P + 16, None) == B.QLORA_ERR_INVALID_ARG   # partial overlap
     with pytest.raises(ValueError):
         B._dropout_args(1.0, 0)
