@@ -173,7 +173,7 @@ def test_finite_differences_for_one_mask():
     X, Wdq, L1, L2, dY = _case(t=3, h=64, o=64, r=16, seed=9)
     p, s = 0.2, 0.5
     keep = O.dropout_keep_mask(3, 64, p, 31337)
-    X64, L164, L264, dY64 = (O._f64(a) for a in (X, L1, L2, dY))
+    X64, L1_64, L2_64, dY64 = (O._f64(a) for a in (X, L1, L2, dY))
     dX, dL1, dL2 = O.qlora_linear_bwd_dropout(dY, X, Wdq, L1, L2, s, keep, p)
 
     def loss(Xv, L1v, L2v):
@@ -185,17 +185,17 @@ def test_finite_differences_for_one_mask():
     for i in range(3):                      # every element of dX, dropped and kept
         for j in range(64):
             E = np.zeros_like(X64); E[i, j] = eps
-            fd = (loss(X64 + E, L164, L264) - loss(X64 - E, L164, L264)) / (2 * eps)
+            fd = (loss(X64 + E, L1_64, L2_64) - loss(X64 - E, L1_64, L2_64)) / (2 * eps)
             assert abs(fd - dX[i, j]) < 1e-7 * (1 + abs(fd))
     rng = np.random.default_rng(0)
     for _ in range(6):
         j = rng.integers(64)
         k, c = rng.integers(64), rng.integers(16)
-        E = np.zeros_like(L164); E[k, c] = eps
-        fd = (loss(X64, L164 + E, L264) - loss(X64, L164 - E, L264)) / (2 * eps)
+        E = np.zeros_like(L1_64); E[k, c] = eps
+        fd = (loss(X64, L1_64 + E, L2_64) - loss(X64, L1_64 - E, L2_64)) / (2 * eps)
         assert abs(fd - dL1[k, c]) < 1e-7 * (1 + abs(fd))
-        E = np.zeros_like(L264); E[c, j] = eps
-        fd = (loss(X64, L164, L264 + E) - loss(X64, L164, L264 - E)) / (2 * eps)
+        E = np.zeros_like(L2_64); E[c, j] = eps
+        fd = (loss(X64, L1_64, L2_64 + E) - loss(X64, L1_64, L2_64 - E)) / (2 * eps)
         assert abs(fd - dL2[c, j]) < 1e-7 * (1 + abs(fd))
 
 
