@@ -1200,15 +1200,14 @@ namespace {
 // One copy per device that loads the library, alive until the process exits.
 static __device__ __align__(256) unsigned char g_static_scratch[QLORA_STATIC_SCRATCH_BYTES];
 
-struct StaticScratch {
-  std::once_flag once;
-  void* ptr = nullptr;  // device address of g_static_scratch on this device
-  int rc = QLORA_ERR_CUDA;
-};
-StaticScratch g_scratch[kMaxDevices];
+// Device address of g_static_scratch per device, cached only once a lookup has succeeded, so
+// that a failed lookup (a transient error, or a first call made during a stream capture) is
+// retried by the next call instead of being remembered.
+std::atomic<void*> g_scratch_ptr[kMaxDevices];
+std::mutex g_scratch_mu;
 
 // In host code the name g_static_scratch is only a host-side stand-in, not a device address:
-// the address a kernel may use is looked up once per device, with that device current.
+// the address a kernel may use is looked up per device, with that device current.
 int static_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -1216,19 +1215,20 @@ int static_scratch(void** out) {
     return QLORA_ERR_CUDA;
   }
   if (dev < 0 || dev >= kMaxDevices) return QLORA_ERR_UNSUPPORTED_DEVICE;
-  StaticScratch& sc = g_scratch[dev];
-  std::call_once(sc.once, [&] {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) {
-      cudaGetLastError();
-      sc.rc = QLORA_ERR_CUDA;
-      return;
+  void* p = g_scratch_ptr[dev].load(std::memory_order_acquire);
+  if (!p) {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    p = g_scratch_ptr[dev].load(std::memory_order_relaxed);
+    if (!p) {
+      if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) {
+        cudaGetLastError();
+        return QLORA_ERR_CUDA;
+      }
+      g_scratch_ptr[dev].store(p, std::memory_order_release);
     }
-    sc.ptr = p;
-    sc.rc = QLORA_OK;
-  });
-  *out = sc.ptr;
-  return sc.rc;
+  }
+  *out = p;
+  return QLORA_OK;
 }
 
 }  // namespace

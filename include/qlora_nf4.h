@@ -164,8 +164,9 @@ QLORA_API int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, int64_t t,
  *   - Arguments and results: exactly those of qlora_linear_fwd without workspace/ws_bytes.
  *   - Limit: shapes with qlora_fwd_workspace_bytes(t, h, o, r) > QLORA_STATIC_SCRATCH_BYTES
  *     are rejected with QLORA_ERR_SCRATCH_LIMIT before anything is launched.
- *   - The first call on a device looks up the array's device address (once per device, with
- *     that device current); make that first call before any stream capture begins.
+ *   - The first call on a device looks up the array's device address (with that device
+ *     current) and keeps it for later calls; make that first call before any stream capture
+ *     begins. A lookup that fails returns QLORA_ERR_CUDA and is tried again by the next call.
  *   - All calls share the one array, and it keeps whatever the previous call left there (the
  *     call clears the parts that must start at zero itself). Two calls whose kernels overlap on
  *     the GPU, for example on two streams, race on the array: serialise them. */

@@ -15,7 +15,7 @@ from bit_quantized_lora_03_b200 import binding as B
 from bit_quantized_lora_03_b200 import inputs
 from oracle import nf4_oracle as O
 
-from gpu_util import assert_close_rms, f32, require_gpu
+from gpu_util import assert_close_rms, f32, oracle_packed_rows, require_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -110,10 +110,39 @@ def test_decode_shape_gemv_4096x11008(t):
     _check_fwd(li)
 
 
-def test_training_shape_linear_sampled():
-    """up_proj of the LLaMA-7B layer (h = 4096, o = 11008, r = 64, t = 4096): full dL1 and
-    dL2, and 256 seeded rows of Y and dX (each row depends on one row of X or dY only)."""
-    li = inputs.training_linear(5)
+@pytest.mark.parametrize("t", [1, 4, 16])
+def test_decode_shape_gemv_8192x28672(t):
+    """The largest decode weight (o x h = 28672 x 8192, 896 row tiles x 128 blocks) through the
+    GEMV at the token counts the bench times: Y on 64 seeded output columns (the oracle
+    quantizes only the scale groups that cover those rows of Wt) and all of sT."""
+    name, Wt = inputs.decode_gemv_weights()[1]
+    o, h = Wt.shape
+    L1, L2 = inputs.decode_gemv_adapters(h, o, 16)
+    X = inputs.decode_gemv_activations(h, t)
+    p = B.nf4_quantize(Wt.cuda())
+    Y, sT = B.qlora_linear_fwd(X.cuda(), p, L1.cuda(), L2.cuda(), 2.0)
+    assert B.last_status() == 0
+    rng = np.random.default_rng(28672 + t)
+    cols = np.unique(np.concatenate([[0, 1, o - 1], rng.choice(o, 61, replace=False)]))
+    Wdq_J = oracle_packed_rows(Wt.numpy(), cols).astype(np.float64)
+    X64, L1_64, L2_64 = f32(X).astype(np.float64), f32(L1).astype(np.float64), f32(L2).astype(np.float64)
+    T = X64 @ L1_64
+    assert_close_rms(f32(sT), 2.0 * T, "sT")
+    Y_ref = X64 @ Wdq_J.T + 2.0 * (T @ L2_64[:, cols])
+    assert_close_rms(f32(Y)[:, cols], Y_ref, "Y columns")
+
+
+@pytest.mark.parametrize("i", [0, 5, 6])
+def test_training_shape_linear_sampled(i):
+    """A training-shape linear of the LLaMA-7B layer (r = 64, t = 4096): q_proj (4096 x 4096:
+    128 CTA-pair tiles, 1.73 waves), up_proj (h = 4096, o = 11008) and down_proj (h = 11008,
+    o = 4096). Full dL1 and dL2, and 256 seeded rows of Y and dX (each row depends on one row
+    of X or dY only). down_proj's dL1 is 11008 x 64: 86 row tiles of 128, between half and all
+    of the 148 SMs, the case the rank-r GEMM plan splits K in two for with two CTAs per SM."""
+    li = inputs.training_linear(i)
+    if i == 6:
+        mtiles = -(-li.h // 128)
+        assert 148 // 2 < mtiles < 148
     p, Y, sT = _run_fwd(li)
     dX, dL1, dL2 = B.qlora_linear_bwd(li.dY.cuda(), li.X.cuda(), p, li.L1.cuda(), li.L2.cuda(),
                                       li.s, sT=sT)
@@ -129,11 +158,14 @@ def test_training_shape_linear_sampled():
     assert_close_rms(f32(dL2), dL2_ref, "dL2")
 
 
-@pytest.mark.parametrize("t,ctas", [(1, 1), (5, 3), (12, 1), (16, 2)])
-def test_decode_gemv_long_warp_runs(t, ctas):
-    """Few CTAs give every warp a long run of units: it crosses row tiles and scale segments
-    (h = 64 x 67: 34 units per row, more than one 32-unit segment, the last unit one block)."""
-    li = inputs.random_linear(t, 64 * 67, 576, 16, 1.5, seed=500 + t, with_grad=False)
+@pytest.mark.parametrize("t,ctas,nblk", [(1, 1, 67), (5, 3, 67), (12, 1, 67), (16, 2, 67),
+                                         (1, 1, 68), (3, 2, 68), (16, 3, 68)])
+def test_decode_gemv_long_warp_runs(t, ctas, nblk):
+    """Few CTAs give every warp a long run of units (32 rows x 128 inputs): it crosses row
+    tiles and 16-unit scale segments. nblk = 67 blocks per row ends every row with a one-block
+    unit and starts rows of 8-bit scales at every byte offset of a 4-byte word; nblk = 68 ends
+    on whole units. Second-level groups of 256 blocks begin in the middle of rows."""
+    li = inputs.random_linear(t, 64 * nblk, 576, 16, 1.5, seed=500 + t + nblk, with_grad=False)
     prev = B.set_gemv_max_ctas(ctas)
     try:
         _check_fwd(li)
