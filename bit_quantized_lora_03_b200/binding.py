@@ -51,6 +51,10 @@ SIGNATURES = {
     "qlora_adamw_step": (ctypes.c_int, [_PTR, _PTR, _PTR, _PTR, _PTR, _I64, ctypes.c_float,
                                         ctypes.c_float, ctypes.c_float, ctypes.c_float,
                                         ctypes.c_float, _I64, ctypes.c_uint, _PTR]),
+    "qlora_adamw_step_multi": (ctypes.c_int, [ctypes.c_int, _PTR, _PTR, _PTR, _PTR, _PTR, _PTR,
+                                              ctypes.c_float, ctypes.c_float, ctypes.c_float,
+                                              ctypes.c_float, ctypes.c_float, _I64, ctypes.c_uint,
+                                              _PTR]),
     "qlora_quantize_codebook": (ctypes.c_int, [_PTR, _PTR, ctypes.c_int, _PTR]),
     "qlora_dequantize_codebook": (ctypes.c_int, [_PTR, ctypes.c_int, _PTR, _PTR]),
     "qlora_quantize_format": (ctypes.c_int, [_PTR, _PTR, ctypes.c_int, ctypes.c_int, _PTR]),
@@ -451,6 +455,48 @@ def adamw_step(p: torch.Tensor, g: torch.Tensor, m: torch.Tensor, v: torch.Tenso
     adamw_step_ptr(p.data_ptr(), p16.data_ptr() if p16 is not None else 0, g.data_ptr(),
                    m.data_ptr(), v.data_ptr(), p.numel(), lr, beta1, beta2, eps, weight_decay,
                    step, 0, stream)
+
+
+ADAMW_MAX_TENSORS = 64
+
+
+def adamw_step_multi_ptr(params, params_bf16, grads, m, v, counts, lr: float, beta1: float,
+                         beta2: float, eps: float, weight_decay: float, step: int, flags: int = 0,
+                         stream=None) -> None:
+    """qlora_adamw_step_multi on lists of raw device pointers (params_bf16 may be None, or hold
+    0 for tensors without a bf16 copy) and parameter counts."""
+    n = len(params)
+    if not (len(grads) == len(m) == len(v) == len(counts) == n) or (
+            params_bf16 is not None and len(params_bf16) != n):
+        raise ValueError("adamw_step_multi: pointer lists of different lengths")
+    P = ctypes.c_void_p * max(n, 1)
+    p16 = P(*params_bf16) if params_bf16 is not None else None
+    _check(lib().qlora_adamw_step_multi(
+        n, P(*params), p16, P(*grads), P(*m), P(*v), (ctypes.c_int64 * max(n, 1))(*counts),
+        float(lr), float(beta1), float(beta2), float(eps), float(weight_decay), int(step),
+        int(flags), _stream(stream)), "qlora_adamw_step_multi")
+
+
+def adamw_step_multi(params, grads, ms, vs, step: int, lr: float = 1e-4, beta1: float = 0.9,
+                     beta2: float = 0.999, eps: float = 1e-8, weight_decay: float = 0.0,
+                     params_bf16=None, stream=None) -> None:
+    """One fused AdamW step over several fp32 CUDA tensors in one launch (in place); each
+    tensor's grad and moments match its shape; params_bf16, if given, is a list holding a bf16
+    tensor (or None) per parameter tensor."""
+    for p, g, m, v in zip(params, grads, ms, vs, strict=True):
+        for t, name in ((p, "p"), (g, "g"), (m, "m"), (v, "v")):
+            _require(t, torch.float32, p.shape, name)
+    ptr16 = None
+    if params_bf16 is not None:
+        ptr16 = []
+        for p, q in zip(params, params_bf16, strict=True):
+            if q is not None:
+                _require(q, torch.bfloat16, p.shape, "p16")
+            ptr16.append(q.data_ptr() if q is not None else 0)
+    adamw_step_multi_ptr([p.data_ptr() for p in params], ptr16, [g.data_ptr() for g in grads],
+                         [m.data_ptr() for m in ms], [v.data_ptr() for v in vs],
+                         [p.numel() for p in params], lr, beta1, beta2, eps, weight_decay, step, 0,
+                         stream)
 
 
 def selftest_wait_timeout(limit_ns: int, stream=None) -> None:

@@ -8,7 +8,8 @@
 //    ("The algebra", mchromiak.github.io; "QLoRA in LLMs" sections 3-4; "The core move",
 //    goodomens.studio: each 4-bit block is dequantized on the fly, used, discarded.)
 //    A (X or dY) and the packed codes arrive by TMA; 8 producer warps turn each 64-weight
-//    block into bf16 (w' = bf16(level * (q8 * s2)), the exact nf4_dequantize values) and
+//    block into bf16 (w' = bf16(level * (q8 * s2)), the exact nf4_dequantize values, selected
+//    by byte permutes from a 16-entry product table built in registers per block) and
 //    write it straight into the 128-byte-swizzled operand layout the MMA reads: K-major for
 //    the forward (rows of Wt are N), MN-major for the backward (rows of Wt are K). A pair of
 //    CTAs (a cluster of 2) owns 512 tokens x 256 columns and issues tcgen05.mma.cta_group::2:
@@ -81,44 +82,74 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// bf16x2 of (a * k, b * k): one packed fp32x2 multiply (IEEE round to nearest per lane, the
-// same two products as two separate multiplies), then round-to-nearest-even to bf16.
-__device__ __forceinline__ uint32_t scale_pack_bf16x2(float a, float b, uint64_t kk) {
-  uint64_t ab, r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(ab) : "f"(a), "f"(b));
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(ab), "l"(kk));
-  float ra, rb;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(ra), "=f"(rb) : "l"(r));
-  return pack_bf16x2(ra, rb);
+// Per-block product table: the 16 exact weights bf16(level[c] * k) of one 64-weight block, held
+// in registers as byte planes so that byte permutes can select them: lo[q] holds the low
+// bytes of entries 4q .. 4q+3, hi[q] their high bytes. Built once per block and stage from the
+// fp32 levels (as eight fp32 pairs) with one packed fp32x2 multiply per pair, so each entry is
+// the value nf4_dequantize produces; no per-weight shared-memory lookup remains.
+struct ProdTab {
+  uint32_t lo[4], hi[4];
+};
+
+__device__ __forceinline__ ProdTab build_prod_tab(const uint64_t (&lv2)[8], float k) {
+  uint64_t kk;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(kk) : "f"(k));
+  uint32_t P[8];   // P[i]: entry 2i in the low half, entry 2i+1 in the high half
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(lv2[i]), "l"(kk));
+    float ra, rb;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(ra), "=f"(rb) : "l"(r));
+    P[i] = pack_bf16x2(ra, rb);
+  }
+  ProdTab t;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    t.lo[q] = __byte_perm(P[2 * q], P[2 * q + 1], 0x6420);
+    t.hi[q] = __byte_perm(P[2 * q], P[2 * q + 1], 0x7531);
+  }
+  return t;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Four weights (codes c_n, n = 0..3; sel: nibble n = c_n & 7; m: byte n = 0xFF if c_n & 8) ->
+// two bf16x2 words (c_0, c_1) and (c_2, c_3), the first of each pair in the low half.
+__device__ __forceinline__ uint2 select4(const ProdTab& t, uint32_t sel, uint32_t m) {
+  const uint32_t L = (prmt(t.lo[0], t.lo[1], sel) & ~m) | (prmt(t.lo[2], t.lo[3], sel) & m);
+  const uint32_t H = (prmt(t.hi[0], t.hi[1], sel) & ~m) | (prmt(t.hi[2], t.hi[3], sel) & m);
+  return make_uint2(prmt(L, H, 0x5140), prmt(L, H, 0x7362));
 }
 
 // Eight packed codes (one 32-bit word, element 2j in the high nibble of byte j) -> eight bf16
-// weights level[code] * k. The level table is 16 fp32 in shared memory; the byte offsets
-// 4*code of all eight nibbles come from two mask operations and one byte-permute each.
-__device__ __forceinline__ uint4 dequant8(uint32_t x, uint64_t kk, const float* lv) {
-  const uint32_t hi4 = (x >> 2) & 0x3C3C3C3Cu;   // byte j: 4 * high nibble
-  const uint32_t lo4 = (x << 2) & 0x3C3C3C3Cu;   // byte j: 4 * low nibble
-  const char* base = reinterpret_cast<const char*>(lv);
-  uint32_t w[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint32_t oh = __byte_perm(hi4, 0u, 0x4440u + j);
-    const uint32_t ol = __byte_perm(lo4, 0u, 0x4440u + j);
-    const float a = *reinterpret_cast<const float*>(base + oh);
-    const float b = *reinterpret_cast<const float*>(base + ol);
-    w[j] = scale_pack_bf16x2(a, b, kk);
-  }
-  return make_uint4(w[0], w[1], w[2], w[3]);
+// weights from the block's product table.
+__device__ __forceinline__ uint4 dequant8(uint32_t x, const ProdTab& t) {
+  const uint32_t x4 = x << 4;   // byte j: the low nibble (element 2j+1) moved up
+  // nibble n = code of element n
+  const uint32_t xs = ((x >> 4) & 0x0F0F0F0Fu) | (x4 & 0xF0F0F0F0u);
+  const uint32_t s = xs & 0x77777777u;
+  // byte n = 0xFF where element n's code has bit 3 set: the sign bit of byte j of x is bit 3 of
+  // element 2j, that of byte j of x4 bit 3 of element 2j+1 (prmt's sign-replicating selectors)
+  const uint32_t m0 = prmt(x, x4, 0xD9C8u);
+  const uint32_t m1 = prmt(x, x4, 0xFBEAu);
+  const uint2 a = select4(t, s, m0);
+  const uint2 b = select4(t, s >> 16, m1);
+  return make_uint4(a.x, a.y, b.x, b.y);
 }
 
 template <bool kBwd>
 __global__ void __launch_bounds__(tc::kThreads, 1)
     nf4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmP,
                     const __grid_constant__ CUtensorMap tmA2,
-                    const __grid_constant__ CUtensorMap tmB2, const Nf4GemmArgs args) {
+                    const __grid_constant__ CUtensorMap tmB2,
+                    const __grid_constant__ CUtensorMap tmOut, const Nf4GemmArgs args) {
   using namespace tc;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ float lv[16];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
@@ -134,9 +165,12 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();             // 0: MMA issuer, 1: its peer
-  const int n0 = blockIdx.y * BN;                        // the pair's 256 output columns
+  // Grid x walks the column tiles (two CTAs each) and grid y the 512-token row blocks, so the
+  // pairs resident at one time share a few row blocks of A (the larger operand) across all
+  // column tiles rather than streaming all of A once per wave.
+  const int n0 = (blockIdx.x >> 1) * BN;                 // the pair's 256 output columns
   const int nh0 = n0 + static_cast<int>(rank) * BNH;    // this CTA's 128 of them
-  const int mrow = (blockIdx.x >> 1) * PAIR_M + static_cast<int>(rank) * 128;  // + a * 256
+  const int mrow = blockIdx.y * PAIR_M + static_cast<int>(rank) * 128;  // + a * 256
   const int total = args.num_kb + args.num_lkb;   // weight K-steps, then the LoRA K-steps
   pdl_launch_dependents();
 
@@ -151,7 +185,6 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     *abort_flag = 0u;
     fence_mbar_init();
   }
-  if (threadIdx.x < 16) lv[threadIdx.x] = args.tab.level[threadIdx.x];
   if (warp == kMmaWarp) {
     tmem_alloc2(tmem_holder, kTmemCols);
     tmem_relinquish2();
@@ -161,6 +194,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     tma_prefetch_desc(&tmP);
     tma_prefetch_desc(&tmA2);
     tma_prefetch_desc(&tmB2);
+    tma_prefetch_desc(&tmOut);
   }
   tc_fence_before();
   __syncthreads();
@@ -260,6 +294,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   } else {
     // ---------------- warps 0-7: dequant producers (half a 64-weight block per thread per
     // stage: 128 blocks of this CTA's 128 columns), then the epilogue -----------------------
+    uint64_t lv2[8];                 // the 16 fp32 levels as pairs (2i low, 2i+1 high)
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      asm("mov.b64 %0, {%1, %2};" : "=l"(lv2[i]) : "f"(args.tab.level[2 * i]), "f"(args.tab.level[2 * i + 1]));
     const int p = threadIdx.x;       // 0..255
     const int blk = p >> 1, half = p & 1;
     const int64_t nblk_row = args.h / kBlock;
@@ -285,69 +323,93 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       out_off = a * 8192 + (jl >> 3) * 1024 + (jl & 7) * 128;
       swz = jl & 7;
     }
-    // 8-bit scale and second-level scale of this thread's block, fetched two stages ahead
+    // 8-bit scale and second-level scale of this thread's block, fetched kPf stages ahead into
+    // a ring of registers; the loop below is unrolled by kPf so that every ring index is a
+    // compile-time constant and a load is waited for only when its stage comes up
+    constexpr int kPf = 4;
     const int nk = args.num_kb;
-    uint32_t q_cur = 0u, q_nxt = 0u;
-    float s_cur = 0.f, s_nxt = 0.f;
-    if (valid && nk > 0) {
-      q_cur = __ldg(args.q8 + qbase);
-      s_cur = __ldg(args.s2 + (qbase >> 8));
-    }
-    if (valid && nk > 1) {
-      const int64_t qi = qbase + qstep;
-      q_nxt = __ldg(args.q8 + qi);
-      s_nxt = __ldg(args.s2 + (qi >> 8));
+    uint32_t qr[kPf];
+    float sr[kPf];
+#pragma unroll
+    for (int j = 0; j < kPf; ++j) {
+      qr[j] = 0u;
+      sr[j] = 0.f;
+      if (valid && j < nk) {
+        const int64_t qi = qbase + static_cast<int64_t>(j) * qstep;
+        qr[j] = __ldg(args.q8 + qi);
+        sr[j] = __ldg(args.s2 + (qi >> 8));
+      }
     }
     bool ok = true;
-    for (int i = 0; i < total && ok; ++i) {
-      const int slot = i % STAGES;
-      const uint32_t ph = (i / STAGES) & 1;
-      if (!mbar_wait(&empty[slot], ph ^ 1u, abort_flag)) { ok = false; break; }
-      if (i < args.num_kb) {
-        const int kb = i;
-        const float k = __fmul_rn(static_cast<float>(q_cur), s_cur);
-        q_cur = q_nxt;
-        s_cur = s_nxt;
-        if (valid && kb + 2 < nk) {
-          const int64_t qi = qbase + static_cast<int64_t>(kb + 2) * qstep;
-          q_nxt = __ldg(args.q8 + qi);
-          s_nxt = __ldg(args.s2 + (qi >> 8));
-        }
-        if (!mbar_wait(&full_ap[slot], ph, abort_flag)) { ok = false; break; }
-        if (valid) {
-          uint64_t kk;
-          asm("mov.b64 %0, {%1, %1};" : "=l"(kk) : "f"(k));
-          const uint4 c = *reinterpret_cast<const uint4*>(sP + slot * P_BYTES + pk_off);
-          const uint32_t words[4] = {c.x, c.y, c.z, c.w};
-          uint8_t* dst = sB + slot * B_BYTES + out_off;
+    for (int i0 = 0; i0 < total && ok; i0 += kPf) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int ch = half * 4 + u;   // 16-byte chunk (8 weights) within the 128-byte row
-            *reinterpret_cast<uint4*>(dst + ((ch ^ swz) << 4)) = dequant8(words[u], kk, lv);
+      for (int j = 0; j < kPf; ++j) {
+        const int i = i0 + j;
+        if (i >= total || !ok) break;
+        const int slot = i % STAGES;
+        const uint32_t ph = (i / STAGES) & 1;
+        if (!mbar_wait(&empty[slot], ph ^ 1u, abort_flag)) { ok = false; break; }
+        if (i < nk) {
+          const float k = __fmul_rn(static_cast<float>(qr[j]), sr[j]);
+          if (valid && i + kPf < nk) {
+            const int64_t qi = qbase + static_cast<int64_t>(i + kPf) * qstep;
+            qr[j] = __ldg(args.q8 + qi);
+            sr[j] = __ldg(args.s2 + (qi >> 8));
           }
+          if (!mbar_wait(&full_ap[slot], ph, abort_flag)) { ok = false; break; }
+          if (valid) {
+            const ProdTab tab = build_prod_tab(lv2, k);
+            const uint4 c = *reinterpret_cast<const uint4*>(sP + slot * P_BYTES + pk_off);
+            const uint32_t words[4] = {c.x, c.y, c.z, c.w};
+            uint8_t* dst = sB + slot * B_BYTES + out_off;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int ch = half * 4 + u;   // 16-byte chunk (8 weights) within the 128-byte row
+              *reinterpret_cast<uint4*>(dst + ((ch ^ swz) << 4)) = dequant8(words[u], tab);
+            }
+          }
+          fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
+        mbar_arrive(&full_b[slot]);
       }
-      mbar_arrive(&full_b[slot]);
     }
 
-    // ---------------- epilogue: TMEM -> registers -> bf16 -> global -------------------------
+    // ---------------- epilogue: TMEM -> registers -> bf16 -> shared -> TMA store -------------
+    // Warp w drains 32 accumulator rows (TMEM lanes 32 (w mod 4) .., accumulator w / 4) in
+    // rounds of 64 columns: four 16-column TMEM loads before one wait, the bf16 row (128 bytes
+    // per lane) into a 32 x 64 staging tile, 128-byte swizzled as the output tensor map
+    // expects (so the eight lanes of each quarter-warp write eight distinct bank groups), then
+    // one TMA store of the tile: whole 128-byte lines instead of 32 scattered row pieces per
+    // store instruction. Two staging tiles per warp (8 KB, in the drained stage buffers) let a
+    // round's shared-memory writes overlap the previous round's store.
     const bool done = mbar_wait(acc_full, 0, abort_flag);
     tc_fence_after();
     if (done && !*abort_flag) {
       if (args.addend) pdl_wait();
       const int acc = warp >> 2, quad = warp & 3;
-      const int row = mrow + acc * 256 + quad * 32 + lane;
+      const int row0 = mrow + acc * 256 + quad * 32;
+      const int row = row0 + lane;
       const uint32_t lane_addr =
           tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      for (int c = 0; c < BN / 16; ++c) {
-        if (n0 + c * 16 >= args.N) break;  // N is a multiple of 64: whole chunks only
-        uint32_t v[16];
-        tmem_ld_16(lane_addr + c * 16, v);
+      uint8_t* stage_tile = smem + warp * 8192;
+      const bool any_row = row0 < args.M;   // warp-uniform: rows past M are not stored
+      // N is a multiple of 64, so a round is either wholly inside the output or wholly past it
+      for (int c0 = 0; c0 < BN / 16; c0 += 4) {
+        if (n0 + c0 * 16 >= args.N) break;
+        uint8_t* buf = stage_tile + ((c0 >> 2) & 1) * 4096;
+        if (c0 >= 8) {   // the store issued from this tile two rounds ago has read it
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
+        }
+        uint32_t vv[4][16];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmem_ld_16(lane_addr + (c0 + q) * 16, vv[q]);
         tmem_ld_wait();
-        if (row < args.M) {
-          const int64_t off = static_cast<int64_t>(row) * args.N + n0 + c * 16;
-          if (args.addend) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t (&v)[16] = vv[q];
+          if (args.addend && row < args.M) {
+            const int64_t off = static_cast<int64_t>(row) * args.N + n0 + (c0 + q) * 16;
             const uint4* ad = reinterpret_cast<const uint4*>(args.addend + off);
             const uint4 a0 = ad[0], a1 = ad[1];
             const uint32_t w[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
@@ -367,11 +429,19 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
           o1.y = pack_bf16x2(__uint_as_float(v[10]), __uint_as_float(v[11]));
           o1.z = pack_bf16x2(__uint_as_float(v[12]), __uint_as_float(v[13]));
           o1.w = pack_bf16x2(__uint_as_float(v[14]), __uint_as_float(v[15]));
-          uint4* dst = reinterpret_cast<uint4*>(args.out + off);
-          dst[0] = o0;
-          dst[1] = o1;
+          uint8_t* rowp = buf + lane * 128;
+          *reinterpret_cast<uint4*>(rowp + (((2 * q) ^ (lane & 7)) << 4)) = o0;
+          *reinterpret_cast<uint4*>(rowp + (((2 * q + 1) ^ (lane & 7)) << 4)) = o1;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && any_row) {
+          tma_store_2d(&tmOut, buf, n0 + c0 * 16, row0);
+          bulk_commit_group();
         }
       }
+      if (lane == 0) bulk_wait_group<0>();   // the output is written before the CTA retires
+      __syncwarp();
     }
   }
   tc_fence_before();

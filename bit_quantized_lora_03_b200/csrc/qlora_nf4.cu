@@ -485,15 +485,20 @@ LoraWs carve_lora(void* base, int64_t, int64_t) {
   return w;
 }
 
-// The fused NF4 GEMM runs as clusters of 2 CTAs (cta_group::2): grid x = 2 CTAs per 512 tokens,
-// grid y = 256-column tiles.
+// The fused NF4 GEMM runs as clusters of 2 CTAs (cta_group::2): grid x = 2 CTAs per 256-column
+// tile, grid y = 512-token row blocks.
 template <bool kBwd>
 int launch_nf4_gemm(const CUtensorMap& mA, const CUtensorMap& mP, const CUtensorMap& mA2,
                     const CUtensorMap& mB2, const Nf4GemmArgs& ga, int64_t t, int64_t ncols,
                     cudaStream_t st, int prof_kind) {
+  // the output (t x ncols bf16) as 32-row x 64-column boxes for the epilogue's TMA stores
+  CUtensorMap mOut;
+  if (!map_bf16(&mOut, ga.out, static_cast<uint64_t>(ncols), static_cast<uint64_t>(t), 64, 32))
+    return QLORA_ERR_CUDA;
+  if ((t + tc::PAIR_M - 1) / tc::PAIR_M > 65535) return QLORA_ERR_BAD_SHAPE;  // grid y limit
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(2 * ((t + tc::PAIR_M - 1) / tc::PAIR_M)),
-                     static_cast<unsigned>((ncols + tc::BN - 1) / tc::BN), 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * ((ncols + tc::BN - 1) / tc::BN)),
+                     static_cast<unsigned>((t + tc::PAIR_M - 1) / tc::PAIR_M), 1);
   cfg.blockDim = dim3(tc::kThreads, 1, 1);
   cfg.dynamicSmemBytes = tc::nf4_gemm_smem_bytes();
   cfg.stream = st;
@@ -511,7 +516,7 @@ int launch_nf4_gemm(const CUtensorMap& mA, const CUtensorMap& mP, const CUtensor
   cudaError_t e;
   {
     prof::Scope ps(prof_kind, st);
-    e = cudaLaunchKernelEx(&cfg, nf4_gemm_kernel<kBwd>, mA, mP, mA2, mB2, ga);
+    e = cudaLaunchKernelEx(&cfg, nf4_gemm_kernel<kBwd>, mA, mP, mA2, mB2, mOut, ga);
   }
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -887,6 +892,59 @@ int qlora_adamw_step(float* param, uint16_t* param_bf16, const float* grad, floa
   return launch_status();
 }
 
+int qlora_adamw_step_multi(int ntensors, float* const* params, uint16_t* const* params_bf16,
+                           const float* const* grads, float* const* m, float* const* v,
+                           const int64_t* counts, float lr, float beta1, float beta2, float eps,
+                           float weight_decay, int64_t step, unsigned flags, qlora_stream_t stream) {
+  if (ntensors < 1 || ntensors > kAdamwMaxTensors || !params || !grads || !m || !v || !counts ||
+      step < 1)
+    return QLORA_ERR_INVALID_ARG;
+  if (!std::isfinite(lr) || !std::isfinite(eps) || !std::isfinite(weight_decay) || eps <= 0.f ||
+      !(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f))
+    return QLORA_ERR_INVALID_ARG;
+  if (flags & ~static_cast<unsigned>(QLORA_ADAMW_PREFETCH)) return QLORA_ERR_INVALID_ARG;
+  AdamwMultiArgs a{};
+  a.ntensors = ntensors;
+  a.first4[0] = 0;
+  for (int k = 0; k < ntensors; ++k) {
+    if (!params[k] || !grads[k] || !m[k] || !v[k] || counts[k] <= 0 || counts[k] % 4 != 0)
+      return QLORA_ERR_INVALID_ARG;
+    uint16_t* p16 = params_bf16 ? params_bf16[k] : nullptr;
+    if (!aligned16(params[k]) || !aligned16(grads[k]) || !aligned16(m[k]) || !aligned16(v[k]) ||
+        (p16 && (reinterpret_cast<uintptr_t>(p16) & 7u)))
+      return QLORA_ERR_MISALIGNED;
+    a.p[k] = params[k];
+    a.p16[k] = p16;
+    a.g[k] = grads[k];
+    a.m[k] = m[k];
+    a.v[k] = v[k];
+    a.first4[k + 1] = a.first4[k] + counts[k] / 4;
+  }
+  int dev, rc;
+  if ((rc = current_device(&dev))) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (flags & QLORA_ADAMW_PREFETCH) {
+    for (int k = 0; k < ntensors; ++k) {
+      const size_t bytes = static_cast<size_t>(counts[k]) * 4;
+      prefetch_if_managed(m[k], bytes, dev, st);
+      prefetch_if_managed(v[k], bytes, dev, st);
+      prefetch_if_managed(params[k], bytes, dev, st);
+      prefetch_if_managed(grads[k], bytes, dev, st);
+    }
+  }
+  a.hy.lr = lr;
+  a.hy.beta1 = beta1;
+  a.hy.beta2 = beta2;
+  a.hy.eps = eps;
+  a.hy.wd = weight_decay;
+  a.hy.step_size = static_cast<float>(lr / (1.0 - std::pow(static_cast<double>(beta1), static_cast<double>(step))));
+  a.hy.inv_sqrt_bc2 = static_cast<float>(1.0 / std::sqrt(1.0 - std::pow(static_cast<double>(beta2), static_cast<double>(step))));
+  const int64_t want = (a.first4[ntensors] + 255) / 256;
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(sm_count(dev)) * 8)));
+  adamw_multi_kernel<<<grid, 256, 0, st>>>(a);
+  return launch_status();
+}
+
 // One thread waits on an mbarrier that no arrival will ever complete; the bounded wait gives
 // up after limit_ns, raises its CTA's abort flag and reports kDevTimeout. Nothing faults.
 __global__ void wait_timeout_selftest_kernel(uint64_t limit_ns) {
@@ -1044,7 +1102,7 @@ int qlora_dequantize_format(const nf4_weight* q, int codebook_id, int scale_form
   if (!aligned16(Wt_out)) return QLORA_ERR_MISALIGNED;
   int dev;
   if ((rc = current_device(&dev))) return rc;
-  const int64_t nitems = q->out_features * q->in_features / 8;
+  const int64_t nitems = q->out_features * q->in_features / 8;   // 8 weights per item
   const int64_t want = (nitems + 4 * 256 - 1) / (4 * 256);
   const int grid = static_cast<int>(std::min<int64_t>(want, int64_t(sm_count(dev)) * 8));
   {

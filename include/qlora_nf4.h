@@ -330,6 +330,19 @@ QLORA_API int qlora_adamw_step(float *param, uint16_t *param_bf16, const float *
                                float eps, float weight_decay, int64_t step, unsigned flags,
                                qlora_stream_t stream);
 
+/* The same AdamW step over several tensors (e.g. all adapters of a layer or a model) in one
+ * launch: tensor k has counts[k] parameters (counts[k] % 4 == 0) at params[k], grads[k], m[k],
+ * v[k] and, if params_bf16 is non-NULL and params_bf16[k] is non-NULL, its bf16 copy at
+ * params_bf16[k]. The pointer arrays and counts are HOST arrays of ntensors entries
+ * (1 <= ntensors <= 64), read before the call returns; the buffers they point to follow the
+ * rules of qlora_adamw_step. Every parameter is updated exactly as qlora_adamw_step updates it
+ * (bit-identical results). Errors as qlora_adamw_step; nothing is launched on an error. */
+QLORA_API int qlora_adamw_step_multi(int ntensors, float *const *params, uint16_t *const *params_bf16,
+                                     const float *const *grads, float *const *m, float *const *v,
+                                     const int64_t *counts, float lr, float beta1, float beta2,
+                                     float eps, float weight_decay, int64_t step, unsigned flags,
+                                     qlora_stream_t stream);
+
 /* Launch shape of the decode GEMV (t <= 16), a scheduling knob with no counterpart in the
  * method. By default the GEMV runs one CTA of 16 warps per SM and splits its units (32 rows x
  * 128 inputs) evenly over all their warps. qlora_set_gemv_max_ctas(n) caps that CTA count at

@@ -157,6 +157,25 @@ def test_adamw_argument_checks(lib):
     assert call(ptr=ctypes.c_void_p(20)) == B.QLORA_ERR_MISALIGNED
 
 
+def test_adamw_multi_argument_checks(lib):
+    f = lib.qlora_adamw_step_multi
+    P = ctypes.c_void_p * 2
+    good = P(16, 32)
+    counts = (ctypes.c_int64 * 2)(64, 128)
+
+    def call(n=2, params=good, grads=good, cnt=counts, step=1, eps=1e-8):
+        return f(n, params, None, grads, good, good, cnt, 1e-3, 0.9, 0.999, eps, 0.0, step, 0, None)
+    assert call(n=0) == B.QLORA_ERR_INVALID_ARG
+    assert call(n=65) == B.QLORA_ERR_INVALID_ARG
+    assert call(params=None) == B.QLORA_ERR_INVALID_ARG
+    assert call(step=0) == B.QLORA_ERR_INVALID_ARG
+    assert call(eps=0.0) == B.QLORA_ERR_INVALID_ARG
+    assert call(grads=P(16, 0)) == B.QLORA_ERR_INVALID_ARG                  # a null entry
+    assert call(cnt=(ctypes.c_int64 * 2)(64, 6)) == B.QLORA_ERR_INVALID_ARG  # count % 4 != 0
+    assert call(cnt=(ctypes.c_int64 * 2)(64, 0)) == B.QLORA_ERR_INVALID_ARG
+    assert call(params=P(16, 36)) == B.QLORA_ERR_MISALIGNED
+
+
 def test_dropout_workspace_and_argument_checks(lib):
     # the dropout calls hold X (.) M (t x h bf16), and the backward also the mask as bits,
     # in front of the plain workspace

@@ -1,6 +1,8 @@
 """GPU parity of qlora_adamw_step (the adapters' update) against the oracle's fp64 AdamW over
 several steps, its bf16 copy bit for bit, and the same step with the optimizer state in unified
-memory (the pages' paged optimizer), also after that state was moved to host memory."""
+memory (the pages' paged optimizer), also after that state was moved to host memory; and
+qlora_adamw_step_multi (all adapters in one launch) against the single-tensor call, bit for bit,
+and against the oracle."""
 
 import ctypes
 
@@ -85,3 +87,49 @@ def test_adamw_with_state_in_unified_memory():
     finally:
         rt.cudaFree(m_ptr)
         rt.cudaFree(v_ptr)
+
+
+def _check_against_oracle(got, ref, name):
+    err = np.abs(got.double().cpu().numpy() - ref)
+    floor = 1e-6 * np.max(np.abs(ref))
+    assert np.all(err <= 4e-6 * np.abs(ref) + floor), f"{name}: max excess {np.max(err - 4e-6 * np.abs(ref) - floor)}"
+
+
+def test_adamw_multi_matches_single_and_oracle():
+    """The 14 adapter tensors of one LLaMA-7B layer at r = 64 (L1 h x r and L2 r x o of seven
+    linears), scaled down in h and o by 8 so the oracle stays quick, plus two tiny tensors of
+    4 and 8 parameters: one multi-tensor launch per step equals 16 single-tensor launches bit
+    for bit (p, m, v and the bf16 copies), over three steps."""
+    require_gpu()
+    shapes = []
+    for h, o in ((512, 512),) * 4 + ((512, 1376),) * 2 + ((1376, 512),):
+        shapes += [(h, 64), (64, o)]
+    shapes += [(4,), (8,)]
+    g0 = torch.Generator().manual_seed(21)
+    p0 = [torch.randn(*sh, generator=g0) * 0.02 for sh in shapes]
+    pa = [x.cuda() for x in p0]
+    pb = [x.cuda() for x in p0]
+    ma, va = [torch.zeros_like(x) for x in pa], [torch.zeros_like(x) for x in pa]
+    mb, vb = [torch.zeros_like(x) for x in pb], [torch.zeros_like(x) for x in pb]
+    qa = [torch.empty_like(x, dtype=torch.bfloat16) if k % 3 else None for k, x in enumerate(pa)]
+    qb = [torch.empty_like(x, dtype=torch.bfloat16) if k % 3 else None for k, x in enumerate(pb)]
+    ref = [(x.double().numpy().ravel(), np.zeros(x.numel()), np.zeros(x.numel())) for x in p0]
+    f = {k: float(np.float32(x)) for k, x in HP.items()}
+    for t in range(1, 4):
+        gs = [torch.randn(*sh, generator=g0) * 0.1 for sh in shapes]
+        gd = [g.cuda() for g in gs]
+        B.adamw_step_multi(pa, gd, ma, va, t, params_bf16=qa, **HP)
+        for k in range(len(shapes)):
+            B.adamw_step(pb[k], gd[k], mb[k], vb[k], t, p16=qb[k], **HP)
+        ref = [O.adamw_step(pr, g.double().numpy().ravel(), mr, vr, t, f["lr"], f["beta1"],
+                            f["beta2"], f["eps"], f["weight_decay"])
+               for (pr, mr, vr), g in zip(ref, gs)]
+    assert B.last_status() == 0
+    torch.cuda.synchronize()
+    for k in range(len(shapes)):
+        assert torch.equal(pa[k], pb[k]) and torch.equal(ma[k], mb[k]) and torch.equal(va[k], vb[k])
+        if qa[k] is not None:
+            assert torch.equal(qa[k], qb[k])
+            assert torch.equal(qa[k], pa[k].to(torch.bfloat16))
+        for got, r, name in zip((pa[k], ma[k], va[k]), ref[k], "pmv"):
+            _check_against_oracle(got.reshape(-1), r, f"{name}[{k}]")
