@@ -80,6 +80,67 @@ __device__ __forceinline__ float fmax_nan(float a, float b) {
   return d;
 }
 
+// Per-block product table: the 16 exact weights bf16(level[c] * k) of one 64-weight block, held
+// in registers as byte planes so that byte permutes can select them: lo[q] holds the low
+// bytes of entries 4q .. 4q+3, hi[q] their high bytes. Built once per block and stage from the
+// fp32 levels (as eight fp32 pairs) with one packed fp32x2 multiply per pair, so each entry is
+// the value nf4_dequantize produces; no per-weight shared-memory lookup remains. Used by the
+// fused GEMM's producers and by the decode GEMV.
+struct ProdTab {
+  uint32_t lo[4], hi[4];
+};
+
+__device__ __forceinline__ ProdTab build_prod_tab(const uint64_t (&lv2)[8], float k) {
+  uint64_t kk;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(kk) : "f"(k));
+  uint32_t P[8];   // P[i]: entry 2i in the low half, entry 2i+1 in the high half
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(lv2[i]), "l"(kk));
+    float ra, rb;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(ra), "=f"(rb) : "l"(r));
+    P[i] = pack_bf16x2(ra, rb);
+  }
+  ProdTab t;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    t.lo[q] = __byte_perm(P[2 * q], P[2 * q + 1], 0x6420);
+    t.hi[q] = __byte_perm(P[2 * q], P[2 * q + 1], 0x7531);
+  }
+  return t;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Four weights (codes c_n, n = 0..3; sel: nibble n = c_n & 7; m: byte n = 0xFF if c_n & 8) ->
+// two bf16x2 words (c_0, c_1) and (c_2, c_3), the first of each pair in the low half.
+__device__ __forceinline__ uint2 select4(const ProdTab& t, uint32_t sel, uint32_t m) {
+  const uint32_t L = (prmt(t.lo[0], t.lo[1], sel) & ~m) | (prmt(t.lo[2], t.lo[3], sel) & m);
+  const uint32_t H = (prmt(t.hi[0], t.hi[1], sel) & ~m) | (prmt(t.hi[2], t.hi[3], sel) & m);
+  return make_uint2(prmt(L, H, 0x5140), prmt(L, H, 0x7362));
+}
+
+// Eight packed codes (one 32-bit word, element 2j in the high nibble of byte j) -> eight bf16
+// weights from the block's product table.
+__device__ __forceinline__ uint4 dequant8_tab(uint32_t x, const ProdTab& t) {
+  const uint32_t x4 = x << 4;   // byte j: the low nibble (element 2j+1) moved up
+  // nibble n = code of element n
+  const uint32_t xs = ((x >> 4) & 0x0F0F0F0Fu) | (x4 & 0xF0F0F0F0u);
+  const uint32_t s = xs & 0x77777777u;
+  // byte n = 0xFF where element n's code has bit 3 set: the sign bit of byte j of x is bit 3 of
+  // element 2j, that of byte j of x4 bit 3 of element 2j+1 (prmt's sign-replicating selectors)
+  const uint32_t m0 = prmt(x, x4, 0xD9C8u);
+  const uint32_t m1 = prmt(x, x4, 0xFBEAu);
+  const uint2 a = select4(t, s, m0);
+  const uint2 b = select4(t, s >> 16, m1);
+  return make_uint4(a.x, a.y, b.x, b.y);
+}
+
 // Persistent: one CTA of 512 threads per SM walks the groups of 256 blocks (16384 weights,
 // 64 KB of fp32) g = blockIdx.x, blockIdx.x + gridDim.x, ...; thread 0 streams each group
 // into one of two 64 KB shared-memory buffers with bulk copies, one group ahead, so HBM reads
