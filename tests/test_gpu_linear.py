@@ -171,3 +171,36 @@ def test_decode_gemv_long_warp_runs(t, ctas, nblk):
         _check_fwd(li)
     finally:
         B.set_gemv_max_ctas(prev)
+
+
+def test_many_tiles_ragged_edges():
+    """More 512 x 256 tiles than CTA pairs fit on the GPU at once (81 in the forward and in the
+    dX kernel), with a ragged last row block (t = 4396 = 8 x 512 + 300) and ragged last column
+    tiles (o = 2176 = 8 x 256 + 128, h = 2112 = 8 x 256 + 64), r = 80 (two LoRA K-steps, the
+    second ragged): Y, sT, dX, dL1 and dL2 in full against the oracle, and the same bits when
+    the call is repeated on a workspace holding other bytes."""
+    t, h, o, r, s = 4396, 2112, 2176, 80, 0.5
+    li = inputs.random_linear(t, h, o, r, s, seed=4396)
+    dev = torch.device("cuda")
+    p = B.nf4_quantize(li.Wt.to(dev))
+    X, dY, L1, L2 = (a.to(dev) for a in (li.X, li.dY, li.L1, li.L2))
+    Wdq = _oracle_weight(li.Wt)
+    Y_ref, sT_ref = O.qlora_linear_fwd(f32(li.X), Wdq, f32(li.L1), f32(li.L2), s)
+    dX_ref, dL1_ref, dL2_ref, _ = O.qlora_linear_bwd(f32(li.dY), f32(li.X), Wdq, f32(li.L1),
+                                                    f32(li.L2), s)
+    outs = []
+    for fill in (0xA5, 0x5A):
+        wsf = torch.full((B.fwd_workspace_bytes(t, h, o, r),), fill, dtype=torch.uint8, device=dev)
+        wsb = torch.full((B.bwd_workspace_bytes(t, h, o, r),), fill, dtype=torch.uint8, device=dev)
+        Y, sT = B.qlora_linear_fwd(X, p, L1, L2, s, ws=wsf)
+        dX, dL1, dL2 = B.qlora_linear_bwd(dY, X, p, L1, L2, s, sT=sT, ws=wsb)
+        torch.cuda.synchronize()
+        assert B.last_status() == 0
+        assert_close_rms(f32(Y), Y_ref, "Y")
+        assert_close_rms(f32(sT), sT_ref, "sT")
+        assert_close_rms(f32(dX), dX_ref, "dX")
+        assert_close_rms(f32(dL1), dL1_ref, "dL1")
+        assert_close_rms(f32(dL2), dL2_ref, "dL2")
+        outs.append((Y.clone(), dX.clone(), dL1.clone(), dL2.clone()))
+    for a_, b_ in zip(*outs):
+        assert torch.equal(a_, b_)
