@@ -196,6 +196,7 @@ __global__ void __launch_bounds__(qz::kThreads, 1) nf4_quantize_kernel(
   float* buf = reinterpret_cast<float*>(qsm);                        // [2][16384]
   uint64_t* full = reinterpret_cast<uint64_t*>(qsm + 2 * qz::kGroupBytes);
   const int tid = threadIdx.x;
+  pdl_launch_dependents();
   if (tid < 16) mids[tid] = tab.mid[tid];
   for (int i = tid; i < 128 * 32; i += qz::kThreads)
     bk[i] = make_float2(bkt.thr[i >> 5], __uint_as_float(static_cast<uint32_t>(bkt.lo[i >> 5])));
@@ -218,6 +219,9 @@ __global__ void __launch_bounds__(qz::kThreads, 1) nf4_quantize_kernel(
     for (uint32_t off = 0; off < bytes; off += qz::kChunk)
       bulk_load(dst + off, src + off, bytes - off < qz::kChunk ? bytes - off : qz::kChunk, &full[b]);
   };
+  // launched with programmatic dependent launch: the set-up above overlaps the kernel before
+  // on the stream, whose completion (and memory) this waits for before any global access
+  pdl_wait();
   if (tid == 0) {
     abort_flag = 0u;
     mbar_init(&full[0], 1);
@@ -291,8 +295,15 @@ __global__ void __launch_bounds__(qz::kThreads, 1) nf4_quantize_kernel(
 }
 
 // Dequantize: each work item is 8 weights (4 packed bytes -> 16 bytes of bf16); a thread
-// takes 4 items spaced a grid apart so that 4 loads are in flight before any compute, and
-// consecutive threads touch consecutive memory (coalesced 4-byte loads, 16-byte stores).
+// takes kDqItems items spaced a grid apart so that that many loads are in flight before any
+// compute, and consecutive threads touch consecutive memory (coalesced 4-byte loads, 16-byte
+// stores). Launched with programmatic dependent launch: the CTAs of a dequantization queued
+// behind another kernel are scheduled while it drains and wait for it before any global
+// access.
+#ifndef QLORA_DQ_ITEMS
+#define QLORA_DQ_ITEMS 4
+#endif
+constexpr int kDqItems = QLORA_DQ_ITEMS;
 __global__ void __launch_bounds__(256) nf4_dequantize_kernel(const uint8_t* __restrict__ codes,
                                                              const uint8_t* __restrict__ q8,
                                                              const float* __restrict__ s2,
@@ -300,15 +311,17 @@ __global__ void __launch_bounds__(256) nf4_dequantize_kernel(const uint8_t* __re
                                                              int64_t nitems, Nf4Table tab,
                                                              int sfmt) {
   __shared__ float lv[16];
+  pdl_launch_dependents();
   if (threadIdx.x < 16) lv[threadIdx.x] = tab.level[threadIdx.x];
   __syncthreads();
+  pdl_wait();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i0 < nitems;
-       i0 += 4 * stride) {
-    uint32_t w[4];
-    float k[4];
+       i0 += kDqItems * stride) {
+    uint32_t w[kDqItems];
+    float k[kDqItems];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kDqItems; ++u) {
       const int64_t it = i0 + u * stride;
       if (it < nitems) {
         w[u] = __ldcs(reinterpret_cast<const unsigned int*>(codes) + it);
@@ -317,7 +330,7 @@ __global__ void __launch_bounds__(256) nf4_dequantize_kernel(const uint8_t* __re
       }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kDqItems; ++u) {
       const int64_t it = i0 + u * stride;
       if (it < nitems) {
         const uint32_t x = w[u];

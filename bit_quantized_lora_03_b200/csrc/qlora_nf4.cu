@@ -1083,11 +1083,26 @@ int qlora_quantize_format(const float* Wt, const nf4_weight* q, int codebook_id,
   const int64_t nblocks = q->out_features * q->in_features / 64;
   const int64_t ngroups = (nblocks + 255) / 256;
   const int grid = static_cast<int>(std::min<int64_t>(ngroups, int64_t(sm_count(dev))));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(qz::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = qz::smem_bytes();
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
   {
     prof::Scope ps(prof::kQuant, reinterpret_cast<cudaStream_t>(stream));
-    nf4_quantize_kernel<<<grid, qz::kThreads, qz::smem_bytes(), reinterpret_cast<cudaStream_t>(stream)>>>(
-        Wt, q->codes, q->absmax_q8, q->absmax_s2, nblocks, device_table(codebook_id),
-        device_buckets(codebook_id), scale_format);
+    e = cudaLaunchKernelEx(&cfg, nf4_quantize_kernel, Wt, q->codes, q->absmax_q8, q->absmax_s2,
+                           nblocks, device_table(codebook_id), device_buckets(codebook_id),
+                           scale_format);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
   }
   return launch_status();
 }
@@ -1103,13 +1118,26 @@ int qlora_dequantize_format(const nf4_weight* q, int codebook_id, int scale_form
   int dev;
   if ((rc = current_device(&dev))) return rc;
   const int64_t nitems = q->out_features * q->in_features / 8;   // 8 weights per item
-  const int64_t want = (nitems + 4 * 256 - 1) / (4 * 256);
+  const int64_t want = (nitems + kDqItems * 256 - 1) / (kDqItems * 256);
   const int grid = static_cast<int>(std::min<int64_t>(want, int64_t(sm_count(dev)) * 8));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(std::max(grid, 1)), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
   {
     prof::Scope ps(prof::kDequant, reinterpret_cast<cudaStream_t>(stream));
-    nf4_dequantize_kernel<<<std::max(grid, 1), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        q->codes, q->absmax_q8, q->absmax_s2, Wt_out, nitems, device_table(codebook_id),
-        scale_format);
+    e = cudaLaunchKernelEx(&cfg, nf4_dequantize_kernel, q->codes, q->absmax_q8, q->absmax_s2,
+                           Wt_out, nitems, device_table(codebook_id), scale_format);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
   }
   return launch_status();
 }
