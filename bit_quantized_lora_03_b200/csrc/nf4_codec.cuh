@@ -141,11 +141,11 @@ __device__ __forceinline__ uint4 dequant8_tab(uint32_t x, const ProdTab& t) {
   return make_uint4(a.x, a.y, b.x, b.y);
 }
 
-// Persistent: one CTA of 512 threads per SM walks the groups of 256 blocks (16384 weights,
-// 64 KB of fp32) g = blockIdx.x, blockIdx.x + gridDim.x, ...; thread 0 streams each group
-// into one of two 64 KB shared-memory buffers with bulk copies, one group ahead, so HBM reads
-// overlap the previous group's arithmetic. Half-warp h of pass p (0..7) owns block 32p + h;
-// each of its lanes reads one float4 of the block from shared memory.
+// Persistent: CTAs of 512 threads (qz::kCtasPerSm per SM) walk the groups of 256 blocks (16384
+// weights, 64 KB of fp32) g = blockIdx.x, blockIdx.x + gridDim.x, ...; thread 0 streams each
+// group into a 64 KB shared-memory buffer with bulk copies, kBufs groups ahead, so HBM reads
+// overlap arithmetic (the other CTA's, with one buffer). Half-warp h of pass p (0..7) owns
+// block 32p + h; each of its lanes reads one float4 of the block from shared memory.
 // 8-bit formats of the block scales ("QLoRA in LLMs" section 1: FP8 E4M3 has 4 exponent and 3
 // fraction bits; section 2 "Choose a scale, then round": symmetric absmax to -127 .. 127). The
 // second level is one fp32 scale s2 per 256 blocks in every format:
@@ -181,10 +181,18 @@ namespace qz {
 constexpr int kThreads = 512;
 constexpr int kGroupBytes = kGroup * kBlock * 4;  // 64 KB
 constexpr int kChunk = 16384;                       // bytes per bulk copy
-constexpr size_t smem_bytes() { return 2 * static_cast<size_t>(kGroupBytes) + 64; }
+#ifndef QLORA_QZ_BUFS
+#define QLORA_QZ_BUFS 1
+#endif
+// Group buffers per CTA. With one, two CTAs share an SM (98 KB of shared memory each): one
+// encodes a group while the other's next group streams in, and 32 warps per SM (not 16)
+// hide the latency of the per-weight shuffles and table lookups.
+constexpr int kBufs = QLORA_QZ_BUFS;
+constexpr int kCtasPerSm = kBufs == 1 ? 2 : 1;
+constexpr size_t smem_bytes() { return kBufs * static_cast<size_t>(kGroupBytes) + 64; }
 }  // namespace qz
 
-__global__ void __launch_bounds__(qz::kThreads, 1) nf4_quantize_kernel(
+__global__ void __launch_bounds__(qz::kThreads, qz::kCtasPerSm) nf4_quantize_kernel(
     const float* __restrict__ W, uint8_t* __restrict__ codes, uint8_t* __restrict__ q8,
     float* __restrict__ s2, int64_t nblocks, Nf4Table tab, Nf4Buckets bkt, int sfmt) {
   extern __shared__ __align__(128) uint8_t qsm[];
@@ -193,8 +201,8 @@ __global__ void __launch_bounds__(qz::kThreads, 1) nf4_quantize_kernel(
   __shared__ float c1s[kGroup];
   __shared__ float wmax[qz::kThreads / 32];
   __shared__ uint32_t abort_flag;
-  float* buf = reinterpret_cast<float*>(qsm);                        // [2][16384]
-  uint64_t* full = reinterpret_cast<uint64_t*>(qsm + 2 * qz::kGroupBytes);
+  float* buf = reinterpret_cast<float*>(qsm);                        // [kBufs][16384]
+  uint64_t* full = reinterpret_cast<uint64_t*>(qsm + qz::kBufs * qz::kGroupBytes);
   const int tid = threadIdx.x;
   pdl_launch_dependents();
   if (tid < 16) mids[tid] = tab.mid[tid];
@@ -224,19 +232,19 @@ __global__ void __launch_bounds__(qz::kThreads, 1) nf4_quantize_kernel(
   pdl_wait();
   if (tid == 0) {
     abort_flag = 0u;
-    mbar_init(&full[0], 1);
-    mbar_init(&full[1], 1);
+    for (int b = 0; b < qz::kBufs; ++b) mbar_init(&full[b], 1);
     fence_mbar_init();
-    if (blockIdx.x < ngroups) issue(blockIdx.x, 0);
-    if (blockIdx.x + gridDim.x < ngroups) issue(blockIdx.x + gridDim.x, 1);
+    for (int b = 0; b < qz::kBufs; ++b)
+      if (blockIdx.x + b * static_cast<int64_t>(gridDim.x) < ngroups)
+        issue(blockIdx.x + b * static_cast<int64_t>(gridDim.x), b);
   }
   __syncthreads();
 
   int it = 0;
   for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x, ++it) {
-    const int b = it & 1;
+    const int b = it % qz::kBufs;
     const int nb = static_cast<int>(group_bytes(g) / (kBlock * 4));
-    if (!mbar_wait(&full[b], static_cast<uint32_t>(it >> 1) & 1u, &abort_flag)) break;
+    if (!mbar_wait(&full[b], static_cast<uint32_t>(it / qz::kBufs) & 1u, &abort_flag)) break;
     const float* gb = buf + b * (kGroup * kBlock);
 #pragma unroll
     for (int p = 0; p < kGroup / 32; ++p) {
@@ -272,9 +280,9 @@ __global__ void __launch_bounds__(qz::kThreads, 1) nf4_quantize_kernel(
       }
     }
     __syncthreads();  // every thread is done with buffer b and has written its c1s
-    if (tid == 0 && g + 2 * static_cast<int64_t>(gridDim.x) < ngroups) {
+    if (tid == 0 && g + qz::kBufs * static_cast<int64_t>(gridDim.x) < ngroups) {
       fence_proxy_async_smem();  // the reads above come before the copy that overwrites b
-      issue(g + 2 * static_cast<int64_t>(gridDim.x), b);
+      issue(g + qz::kBufs * static_cast<int64_t>(gridDim.x), b);
     }
     // second level: c2 = max over the group's block scales; s2 = c2 / top; q8 = code(c1 / s2)
     const float c1 = (tid < nb) ? c1s[tid] : 0.0f;
@@ -295,13 +303,13 @@ __global__ void __launch_bounds__(qz::kThreads, 1) nf4_quantize_kernel(
 }
 
 // Dequantize: each work item is 8 weights (4 packed bytes -> 16 bytes of bf16); a thread
-// takes kDqItems items spaced a grid apart so that that many loads are in flight before any
-// compute, and consecutive threads touch consecutive memory (coalesced 4-byte loads, 16-byte
-// stores). Launched with programmatic dependent launch: the CTAs of a dequantization queued
+// takes kDqItems items spaced a grid apart per round (one measured best: 1 item 0.69, 2 items
+// 0.65, 4 items 0.64, 8 items 0.44 of HBM bandwidth on the LLaMA-7B layer's weights), and
+// consecutive threads touch consecutive memory (coalesced 4-byte loads, 16-byte stores). Launched with programmatic dependent launch: the CTAs of a dequantization queued
 // behind another kernel are scheduled while it drains and wait for it before any global
 // access.
 #ifndef QLORA_DQ_ITEMS
-#define QLORA_DQ_ITEMS 4
+#define QLORA_DQ_ITEMS 1
 #endif
 constexpr int kDqItems = QLORA_DQ_ITEMS;
 __global__ void __launch_bounds__(256) nf4_dequantize_kernel(const uint8_t* __restrict__ codes,

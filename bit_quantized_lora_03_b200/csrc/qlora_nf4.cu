@@ -425,7 +425,8 @@ template <bool A_MN, bool B_MN>
 int launch_tc_gemm(const CUtensorMap& mA, const CUtensorMap& mB, int64_t M, int64_t ncols,
                    const TcPlan& pl, float alpha, int mode, float* out32, int64_t ld,
                    uint16_t* o16a, uint16_t* o16b, int pdl, cudaStream_t st,
-                   const nf4_weight* merge_w = nullptr, const uint8_t* keep_bits = nullptr) {
+                   const nf4_weight* merge_w = nullptr, const uint8_t* keep_bits = nullptr,
+                   const CUtensorMap* mOut = nullptr) {
   TcGemmArgs a{};
   a.M = static_cast<int>(M);
   a.Ncols = static_cast<int>(ncols);
@@ -466,7 +467,8 @@ int launch_tc_gemm(const CUtensorMap& mA, const CUtensorMap& mB, int64_t M, int6
   cudaError_t e;
   {
     prof::Scope ps(prof::kTcGemm, st);
-    e = cudaLaunchKernelEx(&cfg, tc_gemm_kernel<A_MN, B_MN>, mA, mB, a);
+    // the output map is used by the merge epilogue only; the others get A's map as filler
+    e = cudaLaunchKernelEx(&cfg, tc_gemm_kernel<A_MN, B_MN>, mA, mB, mOut ? *mOut : mA, a);
   }
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -830,12 +832,22 @@ int qlora_merge_adapters(const nf4_weight* W, const uint16_t* L1, const uint16_t
   int dev;
   if ((rc = current_device(&dev))) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  CUtensorMap mA, mB;
-  const TcPlan pl = plan_tc(o, h, r, false, sm_count(dev));
-  if (!map_bf16(&mA, L2, o, r, 64, 64) || !map_bf16(&mB, L1, r, h, 64, static_cast<uint32_t>(pl.BNp)))
+  CUtensorMap mA, mB, mOut;
+  TcPlan pl = plan_tc(o, h, r, false, sm_count(dev));
+  pl.splits = 1;   // the merge epilogue needs the whole K (= r) in one CTA
+  pl.kb_per_split = pl.num_kb;
+  // its staging tiles (4 warps x 16 KB) live in the drained stage buffers: keep enough stages
+  while (static_cast<size_t>(pl.stages) * tcg::stage_bytes(pl.BNp, false) < tcg::kMergeStagingBytes &&
+         pl.stages < tcg::MAX_STAGES)
+    ++pl.stages;
+  pl.smem = tcg::smem_bytes(pl.stages, pl.BNp, false);
+  if (static_cast<size_t>(pl.stages) * tcg::stage_bytes(pl.BNp, false) < tcg::kMergeStagingBytes)
+    return QLORA_ERR_BAD_SHAPE;
+  if (!map_bf16(&mA, L2, o, r, 64, 64) || !map_bf16(&mB, L1, r, h, 64, static_cast<uint32_t>(pl.BNp)) ||
+      !make_map_2d(&mOut, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Wt_merged, h, o, h * 4, 32, 32, true))
     return QLORA_ERR_CUDA;
   return launch_tc_gemm<true, false>(mA, mB, o, h, pl, s, kOutMergeNF4, Wt_merged, h, nullptr,
-                                     nullptr, kPdlNone, st, W);
+                                     nullptr, kPdlNone, st, W, nullptr, &mOut);
 }
 
 // Bring a buffer in unified (managed) memory to this device before a kernel touches it, as a
@@ -1082,7 +1094,7 @@ int qlora_quantize_format(const float* Wt, const nf4_weight* q, int codebook_id,
   if ((rc = current_device(&dev))) return rc;
   const int64_t nblocks = q->out_features * q->in_features / 64;
   const int64_t ngroups = (nblocks + 255) / 256;
-  const int grid = static_cast<int>(std::min<int64_t>(ngroups, int64_t(sm_count(dev))));
+  const int grid = static_cast<int>(std::min<int64_t>(ngroups, int64_t(sm_count(dev)) * qz::kCtasPerSm));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
   cfg.blockDim = dim3(qz::kThreads, 1, 1);

@@ -27,6 +27,7 @@ constexpr int kThreads = 6 * 32;            // warps 0-3 epilogue, 4 TMA, 5 MMA
 constexpr int kTmaWarp = 4, kMmaWarp = 5;
 constexpr int kMaxSmem = 232448 - 1024;     // opt-in maximum per CTA on sm_100, less static smem
 constexpr int kSmemPerSm = 233472 - 4096;   // shared memory of one SM, less two CTAs' reserve and static arrays
+constexpr int kMergeStagingBytes = 4 * 16384; // the merge epilogue's staging tiles (4 warps)
 // B tile bytes for a given MMA N (BNp, multiple of 16) and major-ness
 __host__ __device__ constexpr int b_bytes(int BNp, bool b_mn) {
   return b_mn ? ((BNp + 63) / 64) * 8192 : BNp * 128;
@@ -99,7 +100,7 @@ __device__ __forceinline__ void trace_stamp(int slot) {
 template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(tcg::kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const TcGemmArgs args) {
+                   const __grid_constant__ CUtensorMap tmOut, const TcGemmArgs args) {
   using namespace tcg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -309,11 +310,22 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
           *reinterpret_cast<uint4*>(args.out16a + static_cast<int64_t>(grow) * args.Ncols + nb0 + q * 8) = val;
         }
       }
+    } else if (ok && !*abort_flag && args.out_mode == kOutMergeNF4 && STAGES * SB < kMergeStagingBytes) {
+      // the staging tiles must lie inside the drained stage buffers: the host plans enough
+      // stages, and a launch with fewer reports an error instead of writing past them
+      if (lane == 0) report(kDevLaunch);
     } else if (ok && !*abort_flag && args.out_mode == kOutMergeNF4 && args.splits == 1) {
       // 64 columns (one NF4 block of this row) per round: the next block's 32 code bytes and
-      // scales are loaded while this one's accumulator chunks come out of TMEM
+      // scales are loaded while this one's accumulator chunks come out of TMEM. The fp32 row
+      // segment (256 bytes per lane) goes into two 32 x 32 staging tiles, 128-byte swizzled as
+      // the output tensor map expects (the eight lanes of a quarter-warp write eight distinct
+      // bank groups), and two TMA stores write them: whole 128-byte lines rather than 32
+      // scattered 16-byte pieces per store instruction. Two 8 KB staging buffers per warp
+      // (in the drained stage buffers) let a round overlap the previous round's stores.
       const int64_t rowbase = static_cast<int64_t>(row) * args.ld;
       const bool rok = row < args.M;
+      const int row0 = m0 + warp * 32;
+      uint8_t* stg = smem + warp * 16384;
       auto load_block = [&](int col, uint4& ca, uint4& cb, float& k) {
         if (rok && col < args.Ncols) {
           const uint4* src = reinterpret_cast<const uint4*>(args.codes + (rowbase + col) / 2);
@@ -327,6 +339,8 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
       float kk = 0.f;
       load_block(nb0, ca, cb, kk);
       for (int c = 0; c < nchunks; c += 4) {
+        const int col0 = nb0 + c * 16;
+        if (col0 >= args.Ncols) break;   // Ncols % 64 == 0: whole rounds only
         uint32_t v[4][16];
         tmem_ld_16(lane_addr + c * 16, v[0]);
         tmem_ld_16(lane_addr + (c + 1) * 16, v[1]);
@@ -336,27 +350,38 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
         float nk = kk;
         if (c + 4 < nchunks) load_block(nb0 + (c + 4) * 16, na, nbk, nk);
         tmem_ld_wait();
-        const int col0 = nb0 + c * 16;
-        if (rok && col0 < args.Ncols) {
-          const uint32_t words[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
-          float* dst = args.out32 + rowbase + col0;
+        uint8_t* buf = stg + ((c >> 2) & 1) * 8192;
+        if (lane == 0) bulk_wait_group_read<1>();   // the stores two rounds ago have read buf
+        __syncwarp();
+        const uint32_t words[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
 #pragma unroll
-          for (int w = 0; w < 8; ++w) {          // 8 weights per code word
-            float o[8];
+        for (int w = 0; w < 8; ++w) {          // 8 weights per code word
+          float o[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {        // element 2j: high nibble of byte j
-              const uint32_t code = (words[w] >> ((e >> 1) * 8 + ((e & 1) ? 0 : 4))) & 15u;
-              const float wq = __bfloat162float(__float2bfloat16_rn(__fmul_rn(mlv[code], kk)));
-              o[e] = __fadd_rn(wq, __fmul_rn(args.alpha, __uint_as_float(v[w >> 1][(w & 1) * 8 + e])));
-            }
-            *reinterpret_cast<float4*>(dst + 8 * w) = make_float4(o[0], o[1], o[2], o[3]);
-            *reinterpret_cast<float4*>(dst + 8 * w + 4) = make_float4(o[4], o[5], o[6], o[7]);
+          for (int e = 0; e < 8; ++e) {        // element 2j: high nibble of byte j
+            const uint32_t code = (words[w] >> ((e >> 1) * 8 + ((e & 1) ? 0 : 4))) & 15u;
+            const float wq = __bfloat162float(__float2bfloat16_rn(__fmul_rn(mlv[code], kk)));
+            o[e] = __fadd_rn(wq, __fmul_rn(args.alpha, __uint_as_float(v[w >> 1][(w & 1) * 8 + e])));
           }
+          // columns 8w .. 8w+7: tile w / 4, 16-byte chunks 2 (w mod 4) and 2 (w mod 4) + 1
+          uint8_t* rowp = buf + (w >> 2) * 4096 + lane * 128;
+          const int ch = 2 * (w & 3);
+          *reinterpret_cast<float4*>(rowp + ((ch ^ (lane & 7)) << 4)) = make_float4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<float4*>(rowp + (((ch + 1) ^ (lane & 7)) << 4)) = make_float4(o[4], o[5], o[6], o[7]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < args.M) {
+          tma_store_2d(&tmOut, buf, col0, row0);
+          tma_store_2d(&tmOut, buf + 4096, col0 + 32, row0);
+          bulk_commit_group();
         }
         ca = na;
         cb = nbk;
         kk = nk;
       }
+      if (lane == 0) bulk_wait_group<0>();   // the output is written before the CTA retires
+      __syncwarp();
     } else if (ok && !*abort_flag) {
       // up to four 16-column TMEM loads in flight before one wait (the counts are warp-uniform)
       for (int c = 0; c < nchunks; c += 4) {
