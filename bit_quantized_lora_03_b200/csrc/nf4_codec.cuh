@@ -312,6 +312,10 @@ __global__ void __launch_bounds__(qz::kThreads, qz::kCtasPerSm) nf4_quantize_ker
 #define QLORA_DQ_ITEMS 1
 #endif
 constexpr int kDqItems = QLORA_DQ_ITEMS;
+#ifndef QLORA_DQ_CAP
+#define QLORA_DQ_CAP 8
+#endif
+constexpr int kDqCtasPerSm = QLORA_DQ_CAP;   // grid cap: CTAs of 256 threads per SM
 __global__ void __launch_bounds__(256) nf4_dequantize_kernel(const uint8_t* __restrict__ codes,
                                                              const uint8_t* __restrict__ q8,
                                                              const float* __restrict__ s2,

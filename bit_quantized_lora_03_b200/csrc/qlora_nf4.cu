@@ -836,7 +836,9 @@ int qlora_merge_adapters(const nf4_weight* W, const uint16_t* L1, const uint16_t
   TcPlan pl = plan_tc(o, h, r, false, sm_count(dev));
   pl.splits = 1;   // the merge epilogue needs the whole K (= r) in one CTA
   pl.kb_per_split = pl.num_kb;
-  // its staging tiles (4 warps x 16 KB) live in the drained stage buffers: keep enough stages
+  // one stage per K-step (a short K needs no more; a small CTA lets four share an SM), but
+  // the staging tiles (4 warps x 8 KB) live in the drained stage buffers: keep enough stages
+  pl.stages = std::min(pl.num_kb, tcg::MAX_STAGES);
   while (static_cast<size_t>(pl.stages) * tcg::stage_bytes(pl.BNp, false) < tcg::kMergeStagingBytes &&
          pl.stages < tcg::MAX_STAGES)
     ++pl.stages;
@@ -1131,7 +1133,7 @@ int qlora_dequantize_format(const nf4_weight* q, int codebook_id, int scale_form
   if ((rc = current_device(&dev))) return rc;
   const int64_t nitems = q->out_features * q->in_features / 8;   // 8 weights per item
   const int64_t want = (nitems + kDqItems * 256 - 1) / (kDqItems * 256);
-  const int grid = static_cast<int>(std::min<int64_t>(want, int64_t(sm_count(dev)) * 8));
+  const int grid = static_cast<int>(std::min<int64_t>(want, int64_t(sm_count(dev)) * kDqCtasPerSm));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(std::max(grid, 1)), 1, 1);
   cfg.blockDim = dim3(256, 1, 1);

@@ -27,7 +27,7 @@ constexpr int kThreads = 6 * 32;            // warps 0-3 epilogue, 4 TMA, 5 MMA
 constexpr int kTmaWarp = 4, kMmaWarp = 5;
 constexpr int kMaxSmem = 232448 - 1024;     // opt-in maximum per CTA on sm_100, less static smem
 constexpr int kSmemPerSm = 233472 - 4096;   // shared memory of one SM, less two CTAs' reserve and static arrays
-constexpr int kMergeStagingBytes = 4 * 16384; // the merge epilogue's staging tiles (4 warps)
+constexpr int kMergeStagingBytes = 4 * 8192;  // the merge epilogue's staging tiles (4 warps)
 // B tile bytes for a given MMA N (BNp, multiple of 16) and major-ness
 __host__ __device__ constexpr int b_bytes(int BNp, bool b_mn) {
   return b_mn ? ((BNp + 63) / 64) * 8192 : BNp * 128;
@@ -320,12 +320,13 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
       // segment (256 bytes per lane) goes into two 32 x 32 staging tiles, 128-byte swizzled as
       // the output tensor map expects (the eight lanes of a quarter-warp write eight distinct
       // bank groups), and two TMA stores write them: whole 128-byte lines rather than 32
-      // scattered 16-byte pieces per store instruction. Two 8 KB staging buffers per warp
-      // (in the drained stage buffers) let a round overlap the previous round's stores.
+      // scattered 16-byte pieces per store instruction. One 8 KB staging buffer per warp (in
+      // the drained stage buffers) keeps the CTA small: with K = r <= 64 a single stage is
+      // enough, and four CTAs share an SM.
       const int64_t rowbase = static_cast<int64_t>(row) * args.ld;
       const bool rok = row < args.M;
       const int row0 = m0 + warp * 32;
-      uint8_t* stg = smem + warp * 16384;
+      uint8_t* buf = smem + warp * 8192;
       auto load_block = [&](int col, uint4& ca, uint4& cb, float& k) {
         if (rok && col < args.Ncols) {
           const uint4* src = reinterpret_cast<const uint4*>(args.codes + (rowbase + col) / 2);
@@ -350,9 +351,10 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
         float nk = kk;
         if (c + 4 < nchunks) load_block(nb0 + (c + 4) * 16, na, nbk, nk);
         tmem_ld_wait();
-        uint8_t* buf = stg + ((c >> 2) & 1) * 8192;
-        if (lane == 0) bulk_wait_group_read<1>();   // the stores two rounds ago have read buf
-        __syncwarp();
+        if (c > 0) {   // the previous round's stores have read the staging buffer
+          if (lane == 0) bulk_wait_group_read<0>();
+          __syncwarp();
+        }
         const uint32_t words[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
 #pragma unroll
         for (int w = 0; w < 8; ++w) {          // 8 weights per code word
