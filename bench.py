@@ -368,6 +368,23 @@ def codec_leg(dev, peaks):
     }
     del W, packs, outs
     torch.cuda.empty_cache()
+    # one launch long enough for its steady rate: the layer's launches above cover 17-45 M
+    # weights each (6-17 us at the copy bandwidth), where each launch's start and drain
+    # (~2-3 us) weigh in; the 28672 x 8192 decode weight (235 M weights) is one launch
+    o, h = 28672, 8192
+    Wb = inputs.weight_f32(o, h, 301).to(dev)   # the decode recipe's seed for this shape
+    pb = B.PackedNF4(o, h, dev)
+    ob = torch.empty(o, h, dtype=torch.bfloat16, device=dev)
+    qms = queued_ms(lambda: B.nf4_quantize(Wb, out=pb), 5, 2) / 5
+    dms = queued_ms(lambda: B.nf4_dequantize(pb, out=ob), 5, 2) / 5
+    qbytes, dbytes = 4 * o * h + pb.nbytes, pb.nbytes + 2 * o * h
+    res["one_launch_28672x8192"] = {
+        "quantize_ms": round(qms, 4),
+        "quantize_frac_hbm": round(qbytes / (qms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
+        "dequantize_ms": round(dms, 4),
+        "dequantize_frac_hbm": round(dbytes / (dms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)}
+    del Wb, pb, ob
+    torch.cuda.empty_cache()
     return res
 
 
@@ -809,7 +826,7 @@ def decode_case(B, dev, t, wi):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--steps", type=int, default=900)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--tokens", type=int, default=4096)

@@ -302,60 +302,86 @@ __global__ void __launch_bounds__(qz::kThreads, qz::kCtasPerSm) nf4_quantize_ker
   if (bad) report(kDevNonfinite);
 }
 
-// Dequantize: each work item is 8 weights (4 packed bytes -> 16 bytes of bf16); a thread
-// takes kDqItems items spaced a grid apart per round (one measured best: 1 item 0.69, 2 items
-// 0.65, 4 items 0.64, 8 items 0.44 of HBM bandwidth on the LLaMA-7B layer's weights), and
-// consecutive threads touch consecutive memory (coalesced 4-byte loads, 16-byte stores). Launched with programmatic dependent launch: the CTAs of a dequantization queued
-// behind another kernel are scheduled while it drains and wait for it before any global
-// access.
-#ifndef QLORA_DQ_ITEMS
-#define QLORA_DQ_ITEMS 1
-#endif
-constexpr int kDqItems = QLORA_DQ_ITEMS;
-#ifndef QLORA_DQ_CAP
-#define QLORA_DQ_CAP 8
-#endif
-constexpr int kDqCtasPerSm = QLORA_DQ_CAP;   // grid cap: CTAs of 256 threads per SM
-__global__ void __launch_bounds__(256) nf4_dequantize_kernel(const uint8_t* __restrict__ codes,
-                                                             const uint8_t* __restrict__ q8,
-                                                             const float* __restrict__ s2,
-                                                             uint16_t* __restrict__ out,
-                                                             int64_t nitems, Nf4Table tab,
-                                                             int sfmt) {
+// Dequantize, one warp per chunk of 1024 consecutive weights (16 blocks, always inside one
+// group of 256 blocks): each lane loads its 16 code bytes (32 weights, half a block) with one
+// coalesced 16-byte load, the next chunk's codes are loaded before this chunk is converted,
+// and the lane's 64 bytes of bf16 go into a 2 KB staging buffer that one bulk copy
+// (cp.async.bulk, shared -> global) writes out. Two staging buffers per warp alternate, so the
+// warp goes on to its next chunk while the last one's copy drains; the stores are whole lines
+// and cost the threads nothing after the issue. The lanes of a quarter-warp write their 16-byte
+// pieces in a rotated order (lane pairs start at piece 0, 1, 2, 3), so the eight stores of one
+// instruction hit eight distinct bank groups. Launched with programmatic dependent launch: the
+// CTAs of a dequantization queued behind another kernel are scheduled while it drains and wait
+// for it before any global access.
+namespace dq {
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kChunk = 1024;                 // weights per warp per round
+constexpr int kStageBytes = kChunk * 2;      // bf16 of one chunk
+}  // namespace dq
+
+__global__ void __launch_bounds__(dq::kThreads) nf4_dequantize_kernel(const uint8_t* __restrict__ codes,
+                                                                     const uint8_t* __restrict__ q8,
+                                                                     const float* __restrict__ s2,
+                                                                     uint16_t* __restrict__ out,
+                                                                     int64_t n, Nf4Table tab,
+                                                                     int sfmt) {
+  __shared__ __align__(128) uint8_t stage[dq::kWarps][2][dq::kStageBytes];
   __shared__ float lv[16];
   pdl_launch_dependents();
   if (threadIdx.x < 16) lv[threadIdx.x] = tab.level[threadIdx.x];
   __syncthreads();
   pdl_wait();
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i0 < nitems;
-       i0 += kDqItems * stride) {
-    uint32_t w[kDqItems];
-    float k[kDqItems];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t nchunks = (n + dq::kChunk - 1) / dq::kChunk;
+  const int64_t wstride = static_cast<int64_t>(gridDim.x) * dq::kWarps;
+  // this lane's 32 weights of chunk ch: codes and the block scale (two lanes per block)
+  auto load = [&](int64_t ch, uint4& cw, float& k) {
+    const int64_t e0 = ch * dq::kChunk + lane * 32;
+    if (e0 < n) {
+      cw = __ldcs(reinterpret_cast<const uint4*>(codes + e0 / 2));
+      const int64_t b = e0 >> 6;
+      k = __fmul_rn(scale_code_value(__ldg(q8 + b), sfmt), __ldg(s2 + (b >> 8)));
+    }
+  };
+  uint4 cw = make_uint4(0u, 0u, 0u, 0u);
+  float k = 0.f;
+  int64_t ch = static_cast<int64_t>(blockIdx.x) * dq::kWarps + warp;
+  if (ch < nchunks) load(ch, cw, k);
+  for (int round = 0; ch < nchunks; ch += wstride, ++round) {
+    uint4 ncw = cw;
+    float nk = k;
+    if (ch + wstride < nchunks) load(ch + wstride, ncw, nk);
+    uint8_t* buf = stage[warp][round & 1];
+    if (round >= 2) {   // at most one copy (the last round's) may still read its buffer
+      if (lane == 0) bulk_wait_group_read<1>();
+      __syncwarp();
+    }
+    const int64_t base = ch * dq::kChunk;
+    if (base + lane * 32 < n) {
 #pragma unroll
-    for (int u = 0; u < kDqItems; ++u) {
-      const int64_t it = i0 + u * stride;
-      if (it < nitems) {
-        w[u] = __ldcs(reinterpret_cast<const unsigned int*>(codes) + it);
-        const int64_t b = it >> 3;  // 8 items per 64-weight block
-        k[u] = __fmul_rn(scale_code_value(__ldg(q8 + b), sfmt), __ldg(s2 + (b >> 8)));
+      for (int j = 0; j < 4; ++j) {
+        const int q = (j + (lane >> 1)) & 3;   // piece q: weights 8q .. 8q+7 of the lane
+        const uint32_t x = q == 0 ? cw.x : (q == 1 ? cw.y : (q == 2 ? cw.z : cw.w));
+        uint4 o;   // element 2i: high nibble of byte i
+        o.x = pack_bf16x2(__fmul_rn(lv[(x >> 4) & 15u], k), __fmul_rn(lv[x & 15u], k));
+        o.y = pack_bf16x2(__fmul_rn(lv[(x >> 12) & 15u], k), __fmul_rn(lv[(x >> 8) & 15u], k));
+        o.z = pack_bf16x2(__fmul_rn(lv[(x >> 20) & 15u], k), __fmul_rn(lv[(x >> 16) & 15u], k));
+        o.w = pack_bf16x2(__fmul_rn(lv[(x >> 28) & 15u], k), __fmul_rn(lv[(x >> 24) & 15u], k));
+        *reinterpret_cast<uint4*>(buf + lane * 64 + q * 16) = o;
       }
     }
-#pragma unroll
-    for (int u = 0; u < kDqItems; ++u) {
-      const int64_t it = i0 + u * stride;
-      if (it < nitems) {
-        const uint32_t x = w[u];
-        const float kk = k[u];
-        uint4 o;
-        o.x = pack_bf16x2(__fmul_rn(lv[(x >> 4) & 15u], kk), __fmul_rn(lv[x & 15u], kk));
-        o.y = pack_bf16x2(__fmul_rn(lv[(x >> 12) & 15u], kk), __fmul_rn(lv[(x >> 8) & 15u], kk));
-        o.z = pack_bf16x2(__fmul_rn(lv[(x >> 20) & 15u], kk), __fmul_rn(lv[(x >> 16) & 15u], kk));
-        o.w = pack_bf16x2(__fmul_rn(lv[(x >> 28) & 15u], kk), __fmul_rn(lv[(x >> 24) & 15u], kk));
-        __stcs(reinterpret_cast<uint4*>(out) + it, o);
-      }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      const int64_t cnt = n - base < dq::kChunk ? n - base : dq::kChunk;   // a multiple of 64
+      bulk_store(out + base, buf, static_cast<uint32_t>(cnt * 2));
+      bulk_commit_group();
     }
+    cw = ncw;
+    k = nk;
   }
+  if (lane == 0) bulk_wait_group<0>();   // the output is written before the CTA retires
 }
 
 }  // namespace qlora

@@ -211,6 +211,14 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void*
       ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(smem_src)), "r"(x), "r"(y)
       : "memory");
 }
+// Copy `bytes` (a multiple of 16, both addresses 16-byte aligned) from shared to global memory
+// (written by generic stores and made visible with fence_proxy_async_smem first). Tracked by
+// bulk groups like the tensor stores.
+__device__ __forceinline__ void bulk_store(void* gdst, const void* smem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+               ::"l"(reinterpret_cast<uint64_t>(gdst)), "r"(smem_addr(smem_src)), "r"(bytes)
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

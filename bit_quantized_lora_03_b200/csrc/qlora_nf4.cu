@@ -26,6 +26,7 @@ using namespace qlora;
 
 namespace {
 
+constexpr int kMergeCtasPerSm = 4;   // the adapter merge's CTAs per SM (one register bound)
 std::atomic<int> g_gemv_max_ctas{0};  // cap on the decode GEMV's CTAs (0 = one per SM)
 
 // ------------------------------------------------------------------------------------------
@@ -148,6 +149,11 @@ struct DeviceInfo {
   std::once_flag once;
   int ok = 0;        // 1 = sm_100 device ready
   int sms = 148;
+  // CTAs per SM that fit at once (occupancy calculator) for grid-stride kernels whose grids are
+  // one wave of these: a CTA that could only start after others finished would leave SMs idle
+  int dq_ctas = 1;           // nf4_dequantize_kernel
+  int adamw_ctas = 1;        // adamw_kernel, 256 threads
+  int adamw_multi_ctas = 1;  // adamw_multi_kernel, 256 threads
 };
 DeviceInfo g_dev[kMaxDevices];
 
@@ -198,6 +204,18 @@ int current_device(int* dev_out) {
     fine &= cudaFuncSetAttribute(tc_gemm_kernel<true, true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tcg::kMaxSmem) == cudaSuccess;
+    fine &= cudaFuncSetAttribute(tc_gemm_kernel<true, false, kMergeCtasPerSm>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tcg::kMaxSmem) == cudaSuccess;
+    int n = 0;
+    fine &= cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, nf4_dequantize_kernel, dq::kThreads, 0) == cudaSuccess;
+    d.dq_ctas = std::max(1, n);
+    n = 0;
+    fine &= cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, adamw_kernel, 256, 0) == cudaSuccess;
+    d.adamw_ctas = std::max(1, n);
+    n = 0;
+    fine &= cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, adamw_multi_kernel, 256, 0) == cudaSuccess;
+    d.adamw_multi_ctas = std::max(1, n);
     if (!fine) cudaGetLastError();
     d.ok = fine ? 1 : -1;
   });
@@ -207,6 +225,7 @@ int current_device(int* dev_out) {
 }
 
 int sm_count(int dev) { return g_dev[dev].sms; }
+const DeviceInfo& device_info(int dev) { return g_dev[dev]; }
 
 int launch_status() {
   const cudaError_t e = cudaGetLastError();
@@ -421,7 +440,7 @@ TcPlan plan_tc(int64_t M, int64_t ncols, int64_t K, bool b_mn, int sms) {
   return p;
 }
 
-template <bool A_MN, bool B_MN>
+template <bool A_MN, bool B_MN, int kMinCtas = 1>
 int launch_tc_gemm(const CUtensorMap& mA, const CUtensorMap& mB, int64_t M, int64_t ncols,
                    const TcPlan& pl, float alpha, int mode, float* out32, int64_t ld,
                    uint16_t* o16a, uint16_t* o16b, int pdl, cudaStream_t st,
@@ -468,7 +487,7 @@ int launch_tc_gemm(const CUtensorMap& mA, const CUtensorMap& mB, int64_t M, int6
   {
     prof::Scope ps(prof::kTcGemm, st);
     // the output map is used by the merge epilogue only; the others get A's map as filler
-    e = cudaLaunchKernelEx(&cfg, tc_gemm_kernel<A_MN, B_MN>, mA, mB, mOut ? *mOut : mA, a);
+    e = cudaLaunchKernelEx(&cfg, tc_gemm_kernel<A_MN, B_MN, kMinCtas>, mA, mB, mOut ? *mOut : mA, a);
   }
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -567,11 +586,12 @@ size_t keep_bits_bytes(int64_t t, int64_t h) { return align256(static_cast<size_
 // Xd = X (.) M; the keep bits are drawn (and stored into `bits` if given) or, with from_bits,
 // read from `bits`.
 int launch_dropout_apply(const uint16_t* X, int64_t n, uint16_t* Xd, uint8_t* bits, bool from_bits,
-                         const DropoutKey& key, int sms, cudaStream_t st) {
+                         const DropoutKey& key, int dev, cudaStream_t st) {
   const int64_t n8 = n / 8;
   const int64_t per_block = 256 * kDropUnroll;
+  // up to 8 CTAs per SM: more than fit at once (5 or 6), measured ~3% faster than one wave
   const int64_t blocks = std::max<int64_t>(
-      1, std::min<int64_t>((n8 + per_block - 1) / per_block, static_cast<int64_t>(sms) * 8));
+      1, std::min<int64_t>((n8 + per_block - 1) / per_block, static_cast<int64_t>(sm_count(dev)) * 8));
   {
     prof::Scope ps(prof::kDropout, st);
     const auto kern = from_bits ? dropout_apply_kernel<true> : dropout_apply_kernel<false>;
@@ -836,6 +856,8 @@ int qlora_merge_adapters(const nf4_weight* W, const uint16_t* L1, const uint16_t
   TcPlan pl = plan_tc(o, h, r, false, sm_count(dev));
   pl.splits = 1;   // the merge epilogue needs the whole K (= r) in one CTA
   pl.kb_per_split = pl.num_kb;
+  // 128-column tiles: 128 TMEM columns per CTA, so that kMergeCtasPerSm CTAs fit on an SM
+  pl.BNp = static_cast<int>(std::min<int64_t>(128, (h + 15) / 16 * 16));
   // one stage per K-step (a short K needs no more; a small CTA lets four share an SM), but
   // the staging tiles (4 warps x 8 KB) live in the drained stage buffers: keep enough stages
   pl.stages = std::min(pl.num_kb, tcg::MAX_STAGES);
@@ -848,8 +870,9 @@ int qlora_merge_adapters(const nf4_weight* W, const uint16_t* L1, const uint16_t
   if (!map_bf16(&mA, L2, o, r, 64, 64) || !map_bf16(&mB, L1, r, h, 64, static_cast<uint32_t>(pl.BNp)) ||
       !make_map_2d(&mOut, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Wt_merged, h, o, h * 4, 32, 32, true))
     return QLORA_ERR_CUDA;
-  return launch_tc_gemm<true, false>(mA, mB, o, h, pl, s, kOutMergeNF4, Wt_merged, h, nullptr,
-                                     nullptr, kPdlNone, st, W, nullptr, &mOut);
+  return launch_tc_gemm<true, false, kMergeCtasPerSm>(mA, mB, o, h, pl, s, kOutMergeNF4, Wt_merged,
+                                                      h, nullptr, nullptr, kPdlNone, st, W, nullptr,
+                                                      &mOut);
 }
 
 // Bring a buffer in unified (managed) memory to this device before a kernel touches it, as a
@@ -901,7 +924,8 @@ int qlora_adamw_step(float* param, uint16_t* param_bf16, const float* grad, floa
   a.step_size = static_cast<float>(lr / (1.0 - std::pow(static_cast<double>(beta1), static_cast<double>(step))));
   a.inv_sqrt_bc2 = static_cast<float>(1.0 / std::sqrt(1.0 - std::pow(static_cast<double>(beta2), static_cast<double>(step))));
   const int64_t want = (a.n4 + 255) / 256;
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(sm_count(dev)) * 8)));
+  const int grid = static_cast<int>(std::max<int64_t>(
+      1, std::min<int64_t>(want, int64_t(sm_count(dev)) * device_info(dev).adamw_ctas)));
   adamw_kernel<<<grid, 256, 0, st>>>(a);
   return launch_status();
 }
@@ -954,7 +978,8 @@ int qlora_adamw_step_multi(int ntensors, float* const* params, uint16_t* const* 
   a.hy.step_size = static_cast<float>(lr / (1.0 - std::pow(static_cast<double>(beta1), static_cast<double>(step))));
   a.hy.inv_sqrt_bc2 = static_cast<float>(1.0 / std::sqrt(1.0 - std::pow(static_cast<double>(beta2), static_cast<double>(step))));
   const int64_t want = (a.first4[ntensors] + 255) / 256;
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(sm_count(dev)) * 8)));
+  const int grid = static_cast<int>(std::max<int64_t>(
+      1, std::min<int64_t>(want, int64_t(sm_count(dev)) * device_info(dev).adamw_multi_ctas)));
   adamw_multi_kernel<<<grid, 256, 0, st>>>(a);
   return launch_status();
 }
@@ -1131,12 +1156,13 @@ int qlora_dequantize_format(const nf4_weight* q, int codebook_id, int scale_form
   if (!aligned16(Wt_out)) return QLORA_ERR_MISALIGNED;
   int dev;
   if ((rc = current_device(&dev))) return rc;
-  const int64_t nitems = q->out_features * q->in_features / 8;   // 8 weights per item
-  const int64_t want = (nitems + kDqItems * 256 - 1) / (kDqItems * 256);
-  const int grid = static_cast<int>(std::min<int64_t>(want, int64_t(sm_count(dev)) * kDqCtasPerSm));
+  const int64_t n = q->out_features * q->in_features;   // a multiple of 64
+  const int64_t want = (n + dq::kChunk * dq::kWarps - 1) / (dq::kChunk * dq::kWarps);
+  const int grid = static_cast<int>(
+      std::min<int64_t>(want, int64_t(sm_count(dev)) * device_info(dev).dq_ctas));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(std::max(grid, 1)), 1, 1);
-  cfg.blockDim = dim3(256, 1, 1);
+  cfg.blockDim = dim3(dq::kThreads, 1, 1);
   cfg.stream = reinterpret_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1147,7 +1173,7 @@ int qlora_dequantize_format(const nf4_weight* q, int codebook_id, int scale_form
   {
     prof::Scope ps(prof::kDequant, reinterpret_cast<cudaStream_t>(stream));
     e = cudaLaunchKernelEx(&cfg, nf4_dequantize_kernel, q->codes, q->absmax_q8, q->absmax_s2,
-                           Wt_out, nitems, device_table(codebook_id), scale_format);
+                           Wt_out, n, device_table(codebook_id), scale_format);
   }
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -1224,7 +1250,7 @@ int qlora_dropout_apply(const uint16_t* X, int64_t t, int64_t h, float p, uint64
   if (a != b && a < b + bytes && b < a + bytes) return QLORA_ERR_INVALID_ARG;  // partial overlap
   int dev, rc;
   if ((rc = current_device(&dev))) return rc;
-  return launch_dropout_apply(X, t * h, Xd, nullptr, false, dropout_key(p, seed), sm_count(dev),
+  return launch_dropout_apply(X, t * h, Xd, nullptr, false, dropout_key(p, seed), dev,
                               reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -1254,7 +1280,7 @@ int qlora_linear_fwd_dropout(const uint16_t* X, int64_t t, const nf4_weight* W, 
   }
   int dev;
   if ((rc = current_device(&dev))) return rc;
-  if ((rc = launch_dropout_apply(X, t * h, Xd, mask_out, false, key, sm_count(dev), st))) return rc;
+  if ((rc = launch_dropout_apply(X, t * h, Xd, mask_out, false, key, dev, st))) return rc;
   return fwd_core(X, Xd, t, W, L1, L2, r, s_eff, Y, sT_out, rest, st);
 }
 
@@ -1284,7 +1310,7 @@ int qlora_linear_bwd_dropout(const uint16_t* dY, const uint16_t* X, int64_t t, c
   if ((rc = current_device(&dev))) return rc;
   // the forward's mask when given (no generator calls), else drawn again from (p, seed)
   uint8_t* mask = mask_saved ? const_cast<uint8_t*>(mask_saved) : bits;
-  if ((rc = launch_dropout_apply(X, t * h, Xd, mask, mask_saved != nullptr, key, sm_count(dev), st)))
+  if ((rc = launch_dropout_apply(X, t * h, Xd, mask, mask_saved != nullptr, key, dev, st)))
     return rc;
   return bwd_core(dY, Xd, t, W, L1, L2, r, s_eff, sT_saved, dX, dL1, dL2, rest, st, mask, Xd);
 }

@@ -97,8 +97,10 @@ __device__ __forceinline__ void trace_stamp(int slot) {
 #define QLORA_STAMP(i)
 #endif
 
-template <bool A_MN, bool B_MN>
-__global__ void __launch_bounds__(tcg::kThreads, 1)
+// kMinCtas: CTAs that must fit on one SM at once (bounds the registers per thread); the merge
+// runs four small CTAs per SM, the rank-r products one or two large ones.
+template <bool A_MN, bool B_MN, int kMinCtas = 1>
+__global__ void __launch_bounds__(tcg::kThreads, kMinCtas)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmOut, const TcGemmArgs args) {
   using namespace tcg;
@@ -315,49 +317,49 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
       // stages, and a launch with fewer reports an error instead of writing past them
       if (lane == 0) report(kDevLaunch);
     } else if (ok && !*abort_flag && args.out_mode == kOutMergeNF4 && args.splits == 1) {
-      // 64 columns (one NF4 block of this row) per round: the next block's 32 code bytes and
-      // scales are loaded while this one's accumulator chunks come out of TMEM. The fp32 row
-      // segment (256 bytes per lane) goes into two 32 x 32 staging tiles, 128-byte swizzled as
-      // the output tensor map expects (the eight lanes of a quarter-warp write eight distinct
-      // bank groups), and two TMA stores write them: whole 128-byte lines rather than 32
-      // scattered 16-byte pieces per store instruction. One 8 KB staging buffer per warp (in
-      // the drained stage buffers) keeps the CTA small: with K = r <= 64 a single stage is
-      // enough, and four CTAs share an SM.
+      // 32 columns (half an NF4 block of this row) per round: the next round's 16 code bytes
+      // and block scale are loaded while this round's two accumulator chunks come out of TMEM.
+      // The fp32 row segment (128 bytes per lane) goes into a 32 x 32 staging tile, 128-byte
+      // swizzled as the output tensor map expects (the eight lanes of a quarter-warp write
+      // eight distinct bank groups), and one TMA store writes it: whole 128-byte lines rather
+      // than 32 scattered 16-byte pieces per store instruction. Two 4 KB tiles per warp
+      // alternate, so that a round fills one while the store of the round before still reads
+      // the other. They lie in the drained stage buffers (8 KB per warp), and the CTA is small
+      // (one stage, a 128-column tile in 128 TMEM columns, a register bound), so four CTAs
+      // share an SM and one's epilogue overlaps the others' set-up and loads.
       const int64_t rowbase = static_cast<int64_t>(row) * args.ld;
       const bool rok = row < args.M;
       const int row0 = m0 + warp * 32;
       uint8_t* buf = smem + warp * 8192;
-      auto load_block = [&](int col, uint4& ca, uint4& cb, float& k) {
+      auto load_half = [&](int col, uint4& cw, float& k) {
         if (rok && col < args.Ncols) {
-          const uint4* src = reinterpret_cast<const uint4*>(args.codes + (rowbase + col) / 2);
-          ca = src[0];
-          cb = src[1];
+          cw = *reinterpret_cast<const uint4*>(args.codes + (rowbase + col) / 2);
           const int64_t blk = (rowbase + col) / kBlock;
           k = __fmul_rn(static_cast<float>(args.q8[blk]), args.s2[blk / kGroup]);
         }
       };
-      uint4 ca = make_uint4(0u, 0u, 0u, 0u), cb = ca;
+      uint4 cw = make_uint4(0u, 0u, 0u, 0u);
       float kk = 0.f;
-      load_block(nb0, ca, cb, kk);
-      for (int c = 0; c < nchunks; c += 4) {
+      load_half(nb0, cw, kk);
+      for (int c = 0, round = 0; c < nchunks; c += 2, ++round) {
         const int col0 = nb0 + c * 16;
         if (col0 >= args.Ncols) break;   // Ncols % 64 == 0: whole rounds only
-        uint32_t v[4][16];
+        uint32_t v[2][16];
         tmem_ld_16(lane_addr + c * 16, v[0]);
         tmem_ld_16(lane_addr + (c + 1) * 16, v[1]);
-        tmem_ld_16(lane_addr + (c + 2) * 16, v[2]);
-        tmem_ld_16(lane_addr + (c + 3) * 16, v[3]);
-        uint4 na = ca, nbk = cb;
+        uint4 ncw = cw;
         float nk = kk;
-        if (c + 4 < nchunks) load_block(nb0 + (c + 4) * 16, na, nbk, nk);
+        if (c + 2 < nchunks) load_half(nb0 + (c + 2) * 16, ncw, nk);
         tmem_ld_wait();
-        if (c > 0) {   // the previous round's stores have read the staging buffer
-          if (lane == 0) bulk_wait_group_read<0>();
+        uint8_t* tile = buf + (round & 1) * 4096;
+        if (round >= 2) {   // at most one store (the last round's) may still read its tile
+          if (lane == 0) bulk_wait_group_read<1>();
           __syncwarp();
         }
-        const uint32_t words[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+        const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+        uint8_t* rowp = tile + lane * 128;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) {          // 8 weights per code word
+        for (int w = 0; w < 4; ++w) {          // 8 weights per code word
           float o[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {        // element 2j: high nibble of byte j
@@ -365,21 +367,17 @@ __global__ void __launch_bounds__(tcg::kThreads, 1)
             const float wq = __bfloat162float(__float2bfloat16_rn(__fmul_rn(mlv[code], kk)));
             o[e] = __fadd_rn(wq, __fmul_rn(args.alpha, __uint_as_float(v[w >> 1][(w & 1) * 8 + e])));
           }
-          // columns 8w .. 8w+7: tile w / 4, 16-byte chunks 2 (w mod 4) and 2 (w mod 4) + 1
-          uint8_t* rowp = buf + (w >> 2) * 4096 + lane * 128;
-          const int ch = 2 * (w & 3);
-          *reinterpret_cast<float4*>(rowp + ((ch ^ (lane & 7)) << 4)) = make_float4(o[0], o[1], o[2], o[3]);
-          *reinterpret_cast<float4*>(rowp + (((ch + 1) ^ (lane & 7)) << 4)) = make_float4(o[4], o[5], o[6], o[7]);
+          // columns 8w .. 8w+7 of the tile: 16-byte chunks 2w and 2w + 1
+          *reinterpret_cast<float4*>(rowp + (((2 * w) ^ (lane & 7)) << 4)) = make_float4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<float4*>(rowp + (((2 * w + 1) ^ (lane & 7)) << 4)) = make_float4(o[4], o[5], o[6], o[7]);
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0 && row0 < args.M) {
-          tma_store_2d(&tmOut, buf, col0, row0);
-          tma_store_2d(&tmOut, buf + 4096, col0 + 32, row0);
+          tma_store_2d(&tmOut, tile, col0, row0);
           bulk_commit_group();
         }
-        ca = na;
-        cb = nbk;
+        cw = ncw;
         kk = nk;
       }
       if (lane == 0) bulk_wait_group<0>();   // the output is written before the CTA retires
