@@ -644,6 +644,12 @@ int fwd_core(const uint16_t* X, const uint16_t* Xl, int64_t t, const nf4_weight*
     // partial sums of Xl.L1 (+ zeroed sums and counters), then the GEMV, which forms
     // sT = bf16(s . Xl.L1) and finishes Y
     GemvWs gw = carve_gemv(workspace, t, o, r);
+    // codes as 32-row x 64-byte boxes (one unit each); encoded before the first launch, so
+    // that the GEMV's launch follows the LoRA-down kernel's at once and can start under it
+    CUtensorMap mC;
+    if (!make_map_2d(&mC, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, h / 2, o, h / 2, 64,
+                     gv::kTileRows, false))
+      return QLORA_ERR_CUDA;
     {
       prof::Scope ps(prof::kGemvLoraDown, st);
       gemv_lora_down_kernel<<<gd::kCtas, gd::kThreads, gd::smem_bytes(static_cast<int>(t), static_cast<int>(r)), st>>>(
@@ -673,11 +679,6 @@ int fwd_core(const uint16_t* X, const uint16_t* Xl, int64_t t, const nf4_weight*
     const int cap = g_gemv_max_ctas.load(std::memory_order_relaxed);
     if (cap > 0) ctas = std::min<int64_t>(ctas, cap);
     dim3 grid(static_cast<unsigned>(ctas));
-    // codes as 32-row x 64-byte boxes (one unit each)
-    CUtensorMap mC;
-    if (!make_map_2d(&mC, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->codes, h / 2, o, h / 2, 64,
-                     gv::kTileRows, false))
-      return QLORA_ERR_CUDA;
     {
       // programmatic dependent launch: the GEMV's CTAs may start (table, first code loads)
       // while the LoRA-down kernel runs; they wait for its results before using them
