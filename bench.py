@@ -840,6 +840,8 @@ def main():
                     help="with --single-linear: LoRA dropout P on the adapter input")
     ap.add_argument("--gemv-only", action="store_true",
                     help="run only the decode GEMV leg (configuration 3) and print it")
+    ap.add_argument("--codec-only", action="store_true",
+                    help="only the quantize / dequantize leg (the 7B layer's weights, then one long launch)")
     ap.add_argument("--codebooks-only", action="store_true",
                     help="run only the codebook / scale-format comparison leg and print it")
     ap.add_argument("--dropout-only", action="store_true",
@@ -872,6 +874,9 @@ def main():
         return decode_case(B, dev, *args.decode_case)
     if args.codebooks_only:
         print(json.dumps(codebook_leg(dev)), flush=True)
+        return 0
+    if args.codec_only:
+        print(json.dumps(codec_leg(dev, peaks)), flush=True)
         return 0
     if args.gemv_only:
         with ClockSampler(local) as clk:
