@@ -327,10 +327,11 @@ __global__ void __launch_bounds__(dq::kThreads) nf4_dequantize_kernel(const uint
                                                                      int64_t n, Nf4Table tab,
                                                                      int sfmt) {
   __shared__ __align__(128) uint8_t stage[dq::kWarps][2][dq::kStageBytes];
-  __shared__ float lv[16];
   pdl_launch_dependents();
-  if (threadIdx.x < 16) lv[threadIdx.x] = tab.level[threadIdx.x];
-  __syncthreads();
+  uint64_t lv2[8];   // the 16 fp32 levels as pairs (2i low, 2i+1 high)
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    asm("mov.b64 %0, {%1, %2};" : "=l"(lv2[i]) : "f"(tab.level[2 * i]), "f"(tab.level[2 * i + 1]));
   pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t nchunks = (n + dq::kChunk - 1) / dq::kChunk;
@@ -359,16 +360,13 @@ __global__ void __launch_bounds__(dq::kThreads) nf4_dequantize_kernel(const uint
     }
     const int64_t base = ch * dq::kChunk;
     if (base + lane * 32 < n) {
+      // the lane's 32 weights share one block: its 16 exact products, selected by byte permutes
+      const ProdTab pt = build_prod_tab(lv2, k);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int q = (j + (lane >> 1)) & 3;   // piece q: weights 8q .. 8q+7 of the lane
         const uint32_t x = q == 0 ? cw.x : (q == 1 ? cw.y : (q == 2 ? cw.z : cw.w));
-        uint4 o;   // element 2i: high nibble of byte i
-        o.x = pack_bf16x2(__fmul_rn(lv[(x >> 4) & 15u], k), __fmul_rn(lv[x & 15u], k));
-        o.y = pack_bf16x2(__fmul_rn(lv[(x >> 12) & 15u], k), __fmul_rn(lv[(x >> 8) & 15u], k));
-        o.z = pack_bf16x2(__fmul_rn(lv[(x >> 20) & 15u], k), __fmul_rn(lv[(x >> 16) & 15u], k));
-        o.w = pack_bf16x2(__fmul_rn(lv[(x >> 28) & 15u], k), __fmul_rn(lv[(x >> 24) & 15u], k));
-        *reinterpret_cast<uint4*>(buf + lane * 64 + q * 16) = o;
+        *reinterpret_cast<uint4*>(buf + lane * 64 + q * 16) = dequant8_tab(x, pt);
       }
     }
     fence_proxy_async_smem();
