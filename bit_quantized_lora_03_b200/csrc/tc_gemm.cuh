@@ -126,8 +126,6 @@ __global__ void __launch_bounds__(tcg::kThreads, kMinCtas)
   const int b_atoms = (BNp + 63) / 64;
   const uint32_t bbytes = static_cast<uint32_t>(b_bytes(BNp, B_MN));
   pdl_launch_dependents();
-  __shared__ float mlv[16];  // NF4 levels (kOutMergeNF4)
-  if (threadIdx.x < 16) mlv[threadIdx.x] = args.tab.level[threadIdx.x];
 
   if (threadIdx.x == 0) {
     QLORA_STAMP(0);
@@ -312,11 +310,13 @@ __global__ void __launch_bounds__(tcg::kThreads, kMinCtas)
           *reinterpret_cast<uint4*>(args.out16a + static_cast<int64_t>(grow) * args.Ncols + nb0 + q * 8) = val;
         }
       }
-    } else if (ok && !*abort_flag && args.out_mode == kOutMergeNF4 && STAGES * SB < kMergeStagingBytes) {
+    } else if (ok && !*abort_flag && args.out_mode == kOutMergeNF4 &&
+               (kMinCtas == 1 || STAGES * SB < kMergeStagingBytes)) {
+      // the merge runs only in its own instantiation (four CTAs per SM), and
       // the staging tiles must lie inside the drained stage buffers: the host plans enough
       // stages, and a launch with fewer reports an error instead of writing past them
       if (lane == 0) report(kDevLaunch);
-    } else if (ok && !*abort_flag && args.out_mode == kOutMergeNF4 && args.splits == 1) {
+    } else if (kMinCtas > 1 && ok && !*abort_flag && args.out_mode == kOutMergeNF4 && args.splits == 1) {
       // 32 columns (half an NF4 block of this row) per round: the next round's 16 code bytes
       // and block scale are loaded while this round's two accumulator chunks come out of TMEM.
       // The fp32 row segment (128 bytes per lane) goes into a 32 x 32 staging tile, 128-byte
@@ -341,6 +341,10 @@ __global__ void __launch_bounds__(tcg::kThreads, kMinCtas)
       uint4 cw = make_uint4(0u, 0u, 0u, 0u);
       float kk = 0.f;
       load_half(nb0, cw, kk);
+      uint64_t lv2[8];   // the 16 fp32 levels as pairs (2i low, 2i+1 high)
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        asm("mov.b64 %0, {%1, %2};" : "=l"(lv2[i]) : "f"(args.tab.level[2 * i]), "f"(args.tab.level[2 * i + 1]));
       for (int c = 0, round = 0; c < nchunks; c += 2, ++round) {
         const int col0 = nb0 + c * 16;
         if (col0 >= args.Ncols) break;   // Ncols % 64 == 0: whole rounds only
@@ -358,14 +362,18 @@ __global__ void __launch_bounds__(tcg::kThreads, kMinCtas)
         }
         const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
         uint8_t* rowp = tile + lane * 128;
+        // the round's 32 weights share one block: its 16 exact products bf16(level x k),
+        // selected by byte permutes
+        const ProdTab pt = build_prod_tab(lv2, kk);
 #pragma unroll
         for (int w = 0; w < 4; ++w) {          // 8 weights per code word
+          const uint4 b = dequant8_tab(words[w], pt);   // element 2j + 1 in the high half
+          const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
           float o[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {        // element 2j: high nibble of byte j
-            const uint32_t code = (words[w] >> ((e >> 1) * 8 + ((e & 1) ? 0 : 4))) & 15u;
-            const float wq = __bfloat162float(__float2bfloat16_rn(__fmul_rn(mlv[code], kk)));
-            o[e] = __fadd_rn(wq, __fmul_rn(args.alpha, __uint_as_float(v[w >> 1][(w & 1) * 8 + e])));
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t wq = (e & 1) ? (bw[e >> 1] & 0xFFFF0000u) : (bw[e >> 1] << 16);
+            o[e] = __fadd_rn(__uint_as_float(wq), __fmul_rn(args.alpha, __uint_as_float(v[w >> 1][(w & 1) * 8 + e])));
           }
           // columns 8w .. 8w+7 of the tile: 16-byte chunks 2w and 2w + 1
           *reinterpret_cast<float4*>(rowp + (((2 * w) ^ (lane & 7)) << 4)) = make_float4(o[0], o[1], o[2], o[3]);
