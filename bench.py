@@ -647,6 +647,18 @@ def oracle_sample(sample_tokens: int, prepared=None):
     return sample_tokens / total, total, prepared
 
 
+def oracle_sample_one_core(sample_tokens: int, prepared):
+    """The same oracle sample with the BLAS pool limited to one thread (the oracle's other
+    steps are single-threaded numpy already). None if the pool cannot be limited."""
+    try:
+        from threadpoolctl import threadpool_limits
+    except ImportError:
+        return None
+    with threadpool_limits(limits=1):
+        tps, sec, _ = oracle_sample(sample_tokens, prepared)
+    return {"value": round(tps, 3), "unit": UNIT, "cores": 1, "seconds": round(sec, 2)}
+
+
 def cpu_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -1002,11 +1014,14 @@ def main():
                 legs[leg]["cpu_baseline"] = cb
             else:
                 legs[leg + "_cpu_baseline"] = cb
-        tps, sec, _ = oracle_sample(args.cpu_sample_tokens)
+        tps, sec, prepared = oracle_sample(args.cpu_sample_tokens)
         cpu = {"value": round(tps, 3), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                "sample": (f"fwd+bwd of {args.cpu_sample_tokens} of the 4096 tokens, one linear per "
                           "shape class (q 4096x4096 x4, up 4096x11008 x2, down 11008x4096 x1), "
                           f"incl. per-step W dequant; {sec:.1f} s of CPU work")}
+        one = oracle_sample_one_core(args.cpu_sample_tokens, prepared)
+        if one is not None:
+            cpu["one_core"] = one
 
     if rank == 0:
         line = {
