@@ -37,3 +37,22 @@ def test_reference_arm_prints_one_contract_line():
 
 def test_reference_arm_other_ranks_print_nothing():
     assert _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
+
+
+def test_one_core_oracle_sample_runs_with_one_blas_thread(monkeypatch):
+    """The one-core CPU baseline re-times the same prepared sample with the BLAS pool held to
+    one thread, and reports that as its core count."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from threadpoolctl import threadpool_info
+    seen = {}
+
+    def fake_sample(tokens, prepared=None):
+        seen["tokens"], seen["prepared"] = tokens, prepared
+        seen["threads"] = max((d.get("num_threads", 1) for d in threadpool_info()), default=1)
+        return 4.0, 8.0, prepared
+
+    monkeypatch.setattr(bench, "oracle_sample", fake_sample)
+    one = bench.oracle_sample_one_core(32, "prepared-sample")
+    assert seen == {"tokens": 32, "prepared": "prepared-sample", "threads": 1}
+    assert one == {"value": 4.0, "unit": bench.UNIT, "cores": 1, "seconds": 8.0}
