@@ -69,3 +69,26 @@ def test_nf4_has_the_lowest_error_on_normal_weights():
         deq = O.nf4_dequantize_f32(p, O.codebook_levels(cb)).astype(np.float64)
         mse[cb] = float(np.mean((deq - W) ** 2))
     assert mse[0] < mse[1] and mse[0] < mse[2], mse
+
+
+@pytest.mark.parametrize("cb", [1, 2])
+def test_representable_blocks_reproduce_themselves(cb):
+    """A block made of the codebook's own levels times k = q8 * s2 (exact in fp32) keeps its
+    codes and 8-bit scales, and dequantizes to the bf16 rounding of itself, bit for bit. The
+    codes avoid the levels the encoder never chooses: FP4's +0 (a zero weight takes the -0
+    code, the lower of two equal levels) and INT4's -8/7 (below -1)."""
+    q = O.codebook_levels(cb)
+    rng = np.random.default_rng(20 + cb)
+    s2 = np.float32(2.0 ** -8)
+    q8 = np.array([255] + list(rng.integers(1, 256, 255)), np.uint8)
+    k = (q8.astype(np.float32) * s2).astype(np.float32)
+    codes = rng.integers(1, 16, (256, 64)).astype(np.uint8)
+    if cb == 1:
+        codes[codes == 8] = 7
+    codes[:, 0] = 15                      # level +1: every block reaches its absmax exactly
+    W = (q[codes] * k[:, None]).astype(np.float32).reshape(4, 4096)
+    p = O.quantize_with(W, cb)
+    assert np.array_equal(O.unpack_nibbles(p.codes).reshape(256, 64), codes)
+    assert np.array_equal(p.absmax_q8, q8)
+    assert p.absmax_s2[0] == s2
+    assert np.array_equal(O.dequantize_bits_with(p, cb), O.bf16_bits_rne(W))
