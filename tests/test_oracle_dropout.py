@@ -211,3 +211,23 @@ def test_backward_matches_torch_autograd():
     dX, dL1, dL2 = O.qlora_linear_bwd_dropout(dY, X, Wdq, L1, L2, s, keep, p)
     for got, ref in ((dX, tX.grad), (dL1, tL1.grad), (dL2, tL2.grad)):
         assert np.allclose(got, ref.numpy(), rtol=1e-12, atol=1e-14)
+
+
+def test_a_draw_equal_to_the_threshold_is_kept():
+    """The keep rule is draw >= threshold: find an element whose Philox word has its low 8
+    bits zero (so word / 2^32 is exact in fp32), set p to that fraction, and check that the
+    threshold equals the word and that the element is kept."""
+    seed, t, h = 777, 16, 256
+    n = t * h
+    ctr = np.zeros((n // 4, 4), np.uint64)
+    ctr[:, 0] = np.arange(n // 4, dtype=np.uint64)
+    words = O.philox4x32_10(ctr, (seed, 0)).reshape(-1)      # element e takes word e
+    hits = np.nonzero(((words & 0xFF) == 0) & (words > 0))[0]
+    assert hits.size > 0
+    e = int(hits[0])
+    w = int(words[e])
+    p = float(Fraction(w, 2 ** 32))
+    assert float(np.float32(p)) == p and O.dropout_threshold(p) == w
+    keep = O.dropout_keep_mask(t, h, p, seed).reshape(-1)
+    assert keep[e]
+    assert np.array_equal(keep, words.astype(np.int64) >= w)

@@ -196,3 +196,72 @@ def test_unsigned_second_level_matches_textbook_scheme():
         codes, scale = O.absmax_int_quantize(seg, 255, signed=False)
         assert scale == s2[g]
         assert np.array_equal(codes, q8[g * 256:(g + 1) * 256].astype(np.int64))
+
+
+def test_second_level_ties_round_half_to_even():
+    """c1 / s2 exactly halfway between two integers rounds to the even one, as Python's
+    built-in round does: one group whose largest scale is 255 * 2^-8 (so s2 = 2^-8 exactly)
+    and whose other scales are (k + 1/2) * 2^-8, k = 0 .. 254."""
+    c1 = [255.0 * 2.0 ** -8] + [(k + 0.5) * 2.0 ** -8 for k in range(255)]
+    W = np.zeros((256, 64), np.float32)
+    W[:, 0] = np.array(c1, np.float32)
+    W[:, 1] = -0.5 * W[:, 0]              # a second, smaller weight in every block
+    p = O.nf4_quantize(W.reshape(4, 4096))
+    assert p.absmax_s2[0] == np.float32(2.0 ** -8)
+    want = [255] + [round(k + 0.5) for k in range(255)]
+    assert [int(v) for v in p.absmax_q8] == want
+    assert any(w % 2 == 0 and w < k + 0.5 for k, w in enumerate(want[1:]))  # ties went down too
+
+
+def test_dequantize_multiplies_level_by_the_block_scale():
+    """w' = bf16(level * k) with k = fp32(q8 * s2): each product formed exactly in double and
+    rounded once to fp32, then to bf16 by torch's cast. The (level, q8, s2) triples are chosen
+    where the other order, (level * q8) * s2, gives a different bf16 weight, so a swapped order
+    fails; the fp32 values before the bf16 rounding are compared on a random block set too."""
+    import torch
+
+    def bf16_bits(x):
+        return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16) \
+            .view(torch.int16).numpy().view(np.uint16)
+
+    q = O.nf4_codebook()
+    found = []                                   # (s2, q8, code) where the orders differ
+    for seed in range(40):
+        r = np.random.default_rng(seed)
+        s2 = r.uniform(1e-5, 1e-3, 64).astype(np.float32)
+        q8 = r.integers(1, 256, (64, 256)).astype(np.float32)
+        k = (q8.astype(np.float64) * s2[:, None]).astype(np.float32)
+        exact = (q.astype(np.float64)[None, None, :] * k[..., None]).astype(np.float32)
+        other = ((q[None, None, :] * q8[..., None]).astype(np.float32) * s2[:, None, None])
+        i, j, c = np.nonzero(bf16_bits(exact) != bf16_bits(other.astype(np.float32)))
+        found += [(s2[a], int(q8[a, b]), int(cc)) for a, b, cc in zip(i, j, c)]
+        if len(found) >= 8:
+            break
+    assert len(found) >= 8
+    # one group per triple: its first block holds the triple's scale code and only its code
+    ng = len(found)
+    rng = np.random.default_rng(1)
+    codes = rng.integers(0, 16, (ng * 256, 64)).astype(np.uint8)
+    q8 = rng.integers(1, 256, ng * 256).astype(np.uint8)
+    s2 = np.array([f[0] for f in found], np.float32)
+    for g, (_, qq, cc) in enumerate(found):
+        q8[g * 256], codes[g * 256] = qq, cc
+    p = O.NF4Packed(O.pack_nibbles(codes.reshape(-1)), q8, s2, ng * 256, 64, None)
+    k = (q8.astype(np.float64) * s2[np.arange(ng * 256) // 256].astype(np.float64)).astype(np.float32)
+    exact = (q[codes].astype(np.float64) * k[:, None].astype(np.float64)).astype(np.float32)
+    assert np.array_equal(O.nf4_dequantize_f32(p), exact)
+    assert np.array_equal(O.nf4_dequantize_bits(p), bf16_bits(exact))
+
+
+def test_weight_on_a_threshold_takes_the_lower_code():
+    """x = w / c1 equal to a threshold m[i] (the tie of two nearest levels) gives code i, the
+    lower level, and a weight one fp32 step above it gives code i + 1. Blocks have c1 = 1 so
+    that x equals the weight exactly."""
+    mids = O.nf4_midpoints()
+    W = np.zeros((15, 2, 64), np.float32)
+    W[:, :, 0] = 1.0
+    W[:, 0, 1] = mids
+    W[:, 1, 1] = np.nextafter(mids, np.float32(2.0))
+    codes = O.unpack_nibbles(O.nf4_quantize(W.reshape(15, 128)).codes).reshape(15, 2, 64)
+    assert np.array_equal(codes[:, 0, 1], np.arange(15))
+    assert np.array_equal(codes[:, 1, 1], np.arange(1, 16))
