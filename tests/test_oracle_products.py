@@ -132,11 +132,16 @@ def test_backward_against_torch_autograd_float64():
     tW = torch.tensor(Wt, dtype=torch.float64, requires_grad=False)
     tL1 = torch.tensor(L1, dtype=torch.float64, requires_grad=True)
     tL2 = torch.tensor(L2, dtype=torch.float64, requires_grad=True)
-    Y = tX @ tW.T + s * (tX @ tL1) @ tL2
+    T = tX @ tL1
+    T.retain_grad()
+    Y = tX @ tW.T + s * T @ tL2
     Y.backward(torch.tensor(dY, dtype=torch.float64))
-    dX, dL1, dL2, _ = O.qlora_linear_bwd(dY, X, Wt, L1, L2, s)
-    Yo, _ = O.qlora_linear_fwd(X, Wt, L1, L2, s)
+    dX, dL1, dL2, sU = O.qlora_linear_bwd(dY, X, Wt, L1, L2, s)
+    Yo, sT = O.qlora_linear_fwd(X, Wt, L1, L2, s)
     assert np.allclose(Yo, Y.detach().numpy(), rtol=1e-12, atol=1e-12)
+    # the saved rank-r intermediates: sT = s.X.L1 and sU = dY-gradient of T = s.dY.L2^T
+    assert np.allclose(sT, s * T.detach().numpy(), rtol=1e-12, atol=1e-12)
+    assert np.allclose(sU, T.grad.numpy(), rtol=1e-12, atol=1e-12)
     assert np.allclose(dX, tX.grad.numpy(), rtol=1e-12, atol=1e-12)
     assert np.allclose(dL1, tL1.grad.numpy(), rtol=1e-12, atol=1e-12)
     assert np.allclose(dL2, tL2.grad.numpy(), rtol=1e-12, atol=1e-12)

@@ -106,3 +106,44 @@ def test_error_ordering_on_normal_weights():
         d = O.bf16_bits_to_f32(O.dequantize_bits_format(O.quantize_format(W, 0, f), 0, f))
         err.append(float(((d - W) ** 2).mean()))
     assert err[0] < err[1] < err[2]
+
+
+def _bf16_bits(x):
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16) \
+        .view(torch.int16).numpy().view(np.uint16)
+
+
+def test_format_dequantize_multiplies_level_by_the_block_scale():
+    """In every scale format w' = bf16(level * k), k = fp32(value(q8) * s2): the products are
+    formed exactly in double and rounded once (value(q8) has at most 8 significant bits),
+    then cast to bf16 by torch. The (value, s2) pairs are picked where the other order,
+    (level * value) * s2, gives another bf16 weight for some level, so a swapped order fails."""
+    q = O.nf4_codebook()
+    codes_of = {O.SCALES_U8: np.arange(1, 256), O.SCALES_S8: np.arange(1, 128),
+                O.SCALES_E4M3: np.arange(0x08, 0x7F)}
+    for fmt, cand in codes_of.items():
+        vals = O.scale_code_values(cand.astype(np.uint8), fmt).astype(np.float64)
+        found = []                                      # (s2, code byte, level index)
+        for seed in range(5000):
+            s2 = np.float32(np.random.default_rng(seed).uniform(1e-5, 1e-3))
+            k = (vals * np.float64(s2)).astype(np.float32)
+            exact = (q.astype(np.float64)[None, :] * k[:, None]).astype(np.float32)
+            other = ((q[None, :] * vals.astype(np.float32)[:, None]).astype(np.float32) * s2)
+            i, c = np.nonzero(_bf16_bits(exact) != _bf16_bits(other.astype(np.float32)))
+            found += [(s2, int(cand[a]), int(b)) for a, b in zip(i, c)]
+            if len(found) >= 2:
+                break
+        assert len(found) >= 2, fmt
+        ng = len(found)
+        rng = np.random.default_rng(2)
+        codes = rng.integers(0, 16, (ng * 256, 64)).astype(np.uint8)
+        q8 = rng.choice(cand, ng * 256).astype(np.uint8)
+        s2 = np.array([f[0] for f in found], np.float32)
+        for g, (_, qq, cc) in enumerate(found):
+            q8[g * 256], codes[g * 256] = qq, cc
+        p = O.NF4Packed(O.pack_nibbles(codes.reshape(-1)), q8, s2, ng * 256, 64, None)
+        v = O.scale_code_values(q8, fmt).astype(np.float64)
+        k = (v * s2[np.arange(ng * 256) // 256].astype(np.float64)).astype(np.float32)
+        exact = (q[codes].astype(np.float64) * k[:, None].astype(np.float64)).astype(np.float32)
+        got = O.dequantize_bits_format(p, 0, fmt)
+        assert np.array_equal(got, _bf16_bits(exact)), fmt
