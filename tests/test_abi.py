@@ -213,3 +213,17 @@ def test_dropout_workspace_and_argument_checks(lib):
     assert app(P, 4, 128, 0.1, 1, P + 16, None) == B.QLORA_ERR_INVALID_ARG   # partial overlap
     with pytest.raises(ValueError):
         B._dropout_args(1.0, 0)
+
+
+def test_noalloc_forward_rejects_oversized_shapes_on_the_host(lib):
+    """The allocation-free forward refuses, before any CUDA call, a shape whose workspace
+    would not fit its fixed scratch array, and leaves invalid shapes to the forward's own
+    checks (these arguments are never dereferenced)."""
+    P = 0x10000
+    big = _desc(o=1024, h=1024)
+    t, r = 32768, 256                    # sT alone is 32768 x 256 bf16 = 16 MiB
+    assert lib.qlora_fwd_workspace_bytes(t, 1024, 1024, r) > B.QLORA_STATIC_SCRATCH_BYTES
+    f = lib.qlora_linear_fwd_noalloc
+    assert f(P, t, ctypes.byref(big), P, P, r, 1.0, P, None, None) == B.QLORA_ERR_SCRATCH_LIMIT
+    assert f(P, 4, None, P, P, 16, 1.0, P, None, None) == B.QLORA_ERR_INVALID_ARG
+    assert f(P, 4, ctypes.byref(_desc(h=100)), P, P, 16, 1.0, P, None, None) == B.QLORA_ERR_BAD_SHAPE
