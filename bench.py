@@ -85,17 +85,64 @@ def ncu_traffic(kernel: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 50 ms in the background."""
+    """SM clock, power and clock-event reasons of GPU `index` during a timed region: read
+    through NVML every 5 ms by a background thread (a 0.1 s region still gets about twenty
+    samples); where NVML cannot be used, `nvidia-smi -lms 50` in the background instead."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    NVML_PERIOD_S = 0.005
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
         self.path = None
+        self.nvml = None
+        self.rows = []              # NVML samples: (sm MHz, power W, set of reason names)
+        self.max_mhz = None
+        self.stop = None
+        self.thread = None
+
+    def _start_nvml(self):
+        import threading
+        import pynvml as nv
+        nv.nvmlInit()
+        try:
+            h = nv.nvmlDeviceGetHandleByIndex(self.index)   # the index nvidia-smi --id takes
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+
+            def sample():
+                mask = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+                return (float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                        nv.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                        {n for n, b in bits.items() if mask & b})
+            self.rows.append(sample())          # one sample before the region starts
+        except Exception:
+            nv.nvmlShutdown()
+            raise
+        self.nvml = nv
+        self.stop = threading.Event()
+
+        def loop():
+            try:
+                while not self.stop.wait(self.NVML_PERIOD_S):
+                    self.rows.append(sample())
+            except Exception:
+                pass
+        self.thread = threading.Thread(target=loop, daemon=True)
+        self.thread.start()
 
     def __enter__(self):
+        try:
+            self._start_nvml()
+            return self
+        except Exception:
+            self.nvml, self.rows = None, []
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
@@ -108,6 +155,13 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
+        if self.nvml is not None:
+            self.stop.set()
+            self.thread.join(timeout=2.0)
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -117,6 +171,14 @@ class ClockSampler:
         return False
 
     def summary(self):
+        if self.nvml is not None:
+            rows = list(self.rows)
+            if not rows:
+                return None
+            return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": self.max_mhz,
+                    "samples": len(rows),
+                    "reasons": sorted({n for r in rows for n in r[2]}),
+                    "power_w_max": max(r[1] for r in rows), "source": "nvml, every 5 ms"}
         if self.proc is None or not self.path or not os.path.exists(self.path):
             return None
         rows = []
@@ -135,11 +197,12 @@ class ClockSampler:
             except ValueError:
                 return None
         sm = [num(r[1]) for r in rows if num(r[1]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        reasons = sorted({n for r in rows for n, v in zip(self.REASONS, r[5:9])
+                          if v.lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": num(rows[0][2]), "samples": len(rows), "reasons": reasons,
-                "power_w_max": max((num(r[3]) or 0.0) for r in rows)}
+                "power_w_max": max((num(r[3]) or 0.0) for r in rows),
+                "source": "nvidia-smi, every 50 ms"}
 
 
 # ------------------------------------------------------------------------------------------

@@ -56,3 +56,65 @@ def test_one_core_oracle_sample_runs_with_one_blas_thread(monkeypatch):
     one = bench.oracle_sample_one_core(32, "prepared-sample")
     assert seen == {"tokens": 32, "prepared": "prepared-sample", "threads": 1}
     assert one == {"value": 4.0, "unit": bench.UNIT, "cores": 1, "seconds": 8.0}
+
+
+class _FakeNvml:
+    """Stands in for pynvml: SM clock cycles 1700, 1800, 1900 MHz, 900 W, power cap active."""
+    NVML_CLOCK_SM = 1
+    nvmlClocksEventReasonSwPowerCap = 0x4
+    nvmlClocksEventReasonHwSlowdown = 0x8
+    nvmlClocksEventReasonSwThermalSlowdown = 0x20
+    nvmlClocksEventReasonHwThermalSlowdown = 0x40
+
+    def __init__(self, fail_init=False):
+        self.fail_init, self.n, self.shut = fail_init, 0, False
+
+    def nvmlInit(self):
+        if self.fail_init:
+            raise RuntimeError("no NVML")
+
+    def nvmlShutdown(self):
+        self.shut = True
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return ("gpu", i)
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        assert kind == self.NVML_CLOCK_SM
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        assert kind == self.NVML_CLOCK_SM
+        self.n += 1
+        return (1700, 1800, 1900)[self.n % 3]
+
+    def nvmlDeviceGetPowerUsage(self, h):
+        return 900_000                                  # mW
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return 0x4 | 0x1                               # power cap + idle bit (not reported)
+
+
+def test_clock_sampler_reads_nvml_during_the_region(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import time
+    import bench
+    fake = _FakeNvml()
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    with bench.ClockSampler(0) as clk:
+        time.sleep(0.1)
+    s = clk.summary()
+    assert fake.shut and s["source"].startswith("nvml")
+    assert s["samples"] >= 5 and s["sm_mhz"] in (1700.0, 1800.0, 1900.0)
+    assert s["sm_max_mhz"] == 1965.0 and s["power_w_max"] == 900.0
+    assert s["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_sampler_falls_back_when_nvml_is_missing(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setitem(sys.modules, "pynvml", _FakeNvml(fail_init=True))
+    monkeypatch.setenv("PATH", "/nonexistent")      # and no nvidia-smi either: no record
+    with bench.ClockSampler(0) as clk:
+        pass
+    assert clk.nvml is None and clk.summary() is None
