@@ -38,8 +38,8 @@ Readings where the pages are silent (each is also listed in the design notes):
   8 positive quantiles at probabilities evenly spaced from delta down to (not including)
   1/2, 7 negative ones likewise, the zero, all divided by the largest; delta is the mean of
   the two "centre of the outermost of 15 / of 16 equal-probability bins" probabilities,
-  1 - 1/30 and 1 - 1/32. The exact delta is a reading: parity of the 16 values is pinned
-  by the properties above, not by a printed table (the pages print none).
+  1 - 1/30 and 1 - 1/32. The exact delta is a reading, so the exact 16 values are parity
+  unpinned beyond the properties above: no printed table pins them (the pages print none).
 * Code choice: nearest level by comparison against fp32 midpoints of adjacent levels; a
   value exactly on a midpoint takes the lower code.
 * Second level: unsigned 8-bit absmax codes with step c2/255 (the textbook scheme of
