@@ -32,6 +32,17 @@ def _bits(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().view(torch.int16).numpy().astype(np.uint16)
 
 
+def _tie_p(t: int, h: int, seed: int) -> float:
+    """A dropout probability whose threshold equals one of the draws of this (t, h, seed):
+    the first word with its low 8 bits zero, over 2^32 (exact in fp32)."""
+    n = t * h
+    ctr = np.zeros((n // 4, 4), np.uint64)
+    ctr[:, 0] = np.arange(n // 4, dtype=np.uint64)
+    words = O.philox4x32_10(ctr, (seed, 0)).reshape(-1)
+    w = int(words[np.nonzero(((words & 0xFF) == 0) & (words > 0))[0][0]])
+    return w / 2.0 ** 32
+
+
 @pytest.mark.parametrize("t,h,p,seed", [
     (1, 64, 0.05, 0),
     (37, 320, 0.5, 123),
@@ -39,6 +50,7 @@ def _bits(t: torch.Tensor) -> np.ndarray:
     (5, 128, 0.0, 9),                   # p = 0 keeps everything
     (64, 640, 0.9, (1 << 64) - 1),
     (3, 64, 1e-12, 4),                  # below 2^-32: threshold 0
+    (16, 256, _tie_p(16, 256, 777), 777),  # one draw equals the threshold: that element is kept
 ])
 def test_dropout_mask_bit_exact(t, h, p, seed):
     X = inputs.normal_bf16((t, h), 1.0, inputs._gen(900 + t))
