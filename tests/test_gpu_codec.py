@@ -164,3 +164,13 @@ def test_other_scale_formats_bit_exact(cb, fmt):
     W[20:40] *= 1e-5          # block scales far below the group's largest: E4M3 subnormals
     W[160:] = 0.0             # blocks 480 .. 770 zero: second-level group 2 entirely zero
     _check_format(W, cb, fmt)
+
+
+def test_second_level_ties_round_half_to_even():
+    """Block scales with c1 / s2 exactly halfway between two integers (s2 = 2^-8 exactly, c1 =
+    (k + 1/2) 2^-8): the 8-bit codes round half to even on the GPU as in the oracle."""
+    c1 = [255.0 * 2.0 ** -8] + [(k + 0.5) * 2.0 ** -8 for k in range(255)]
+    W = torch.zeros(256, 64)
+    W[:, 0] = torch.tensor(c1, dtype=torch.float32)
+    W[:, 1] = -0.5 * W[:, 0]
+    _check_full(W.reshape(4, 4096))
