@@ -174,3 +174,37 @@ def test_second_level_ties_round_half_to_even():
     W[:, 0] = torch.tensor(c1, dtype=torch.float32)
     W[:, 1] = -0.5 * W[:, 0]
     _check_full(W.reshape(4, 4096))
+
+
+def test_dequantize_where_the_multiply_order_matters():
+    """Packed weights whose (level, q8, s2) make (level * q8) * s2 and level * (q8 * s2) round
+    to different bf16 values: the GPU dequantizer gives the second, as the oracle does."""
+    q = O.nf4_codebook()
+    found = []
+    for seed in range(40):
+        r = np.random.default_rng(seed)
+        s2 = r.uniform(1e-5, 1e-3, 64).astype(np.float32)
+        q8 = r.integers(1, 256, (64, 256)).astype(np.float32)
+        k = (q8 * s2[:, None]).astype(np.float32)
+        exact = (q[None, None, :] * k[..., None]).astype(np.float32)
+        other = ((q[None, None, :] * q8[..., None]).astype(np.float32) * s2[:, None, None])
+        i, j, c = np.nonzero(O.bf16_bits_rne(exact) != O.bf16_bits_rne(other.astype(np.float32)))
+        found += [(s2[a], int(q8[a, b]), int(cc)) for a, b, cc in zip(i, j, c)]
+        if len(found) >= 8:
+            break
+    assert len(found) >= 8
+    ng = len(found)
+    rng = np.random.default_rng(3)
+    codes = rng.integers(0, 16, (ng * 256, 64)).astype(np.uint8)
+    q8 = rng.integers(1, 256, ng * 256).astype(np.uint8)
+    s2 = np.array([f[0] for f in found], np.float32)
+    for g, (_, qq, cc) in enumerate(found):
+        q8[g * 256], codes[g * 256] = qq, cc
+    ref = O.NF4Packed(O.pack_nibbles(codes.reshape(-1)), q8, s2, ng * 256, 64, None)
+    p = B.PackedNF4(ng * 256, 64, "cuda")
+    p.codes.copy_(torch.from_numpy(ref.codes))
+    p.absmax_q8.copy_(torch.from_numpy(q8))
+    p.absmax_s2.copy_(torch.from_numpy(s2))
+    got = B.nf4_dequantize(p).view(torch.int16).cpu().numpy().view(np.uint16)
+    assert B.last_status() == 0
+    assert np.array_equal(got, O.nf4_dequantize_bits(ref))
