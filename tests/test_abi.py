@@ -227,3 +227,17 @@ def test_noalloc_forward_rejects_oversized_shapes_on_the_host(lib):
     assert f(P, t, ctypes.byref(big), P, P, r, 1.0, P, None, None) == B.QLORA_ERR_SCRATCH_LIMIT
     assert f(P, 4, None, P, P, 16, 1.0, P, None, None) == B.QLORA_ERR_INVALID_ARG
     assert f(P, 4, ctypes.byref(_desc(h=100)), P, P, 16, 1.0, P, None, None) == B.QLORA_ERR_BAD_SHAPE
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch):
+    """No CPU or library fallback: with the library missing every call raises, and a host
+    tensor is refused rather than computed on the CPU."""
+    import torch
+    monkeypatch.setattr(B, "_lib", None)
+    monkeypatch.setattr(B, "library_path", lambda: os.path.join(ROOT, "no-such-dir", "lib.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        B.lib()
+    with pytest.raises((RuntimeError, ValueError)):
+        B.nf4_quantize(torch.zeros(4, 64))
+    with pytest.raises((RuntimeError, ValueError)):
+        B.nf4_dequantize(B.PackedNF4(4, 64, "cpu"))
