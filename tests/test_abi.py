@@ -86,8 +86,8 @@ def test_host_validation_rejects_before_launch(lib):
     assert lib.nf4_quantize(0x1000, ctypes.byref(bad_h), None) == B.QLORA_ERR_BAD_SHAPE
     zero_o = _desc(o=0)
     assert lib.nf4_quantize(0x1000, ctypes.byref(zero_o), None) == B.QLORA_ERR_BAD_SHAPE
-    mis = _desc(codes=0x1001)
-    assert lib.nf4_quantize(0x1000, ctypes.byref(mis), None) == B.QLORA_ERR_MISALIGNED
+    for mis in (_desc(codes=0x1001), _desc(q8=0x2008), _desc(s2=0x3004)):
+        assert lib.nf4_quantize(0x1000, ctypes.byref(mis), None) == B.QLORA_ERR_MISALIGNED
     assert lib.nf4_quantize(0x1004, ctypes.byref(d), None) == B.QLORA_ERR_MISALIGNED
     null_codes = _desc(codes=0)
     assert lib.nf4_dequantize(ctypes.byref(null_codes), 0x1000, None) == B.QLORA_ERR_INVALID_ARG
