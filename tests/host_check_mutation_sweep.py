@@ -71,8 +71,8 @@ def run(name, tmp):
                         "-p", "no:cacheprovider"], cwd=d, capture_output=True, text=True,
                        timeout=900)
     failed = [line for line in r.stdout.splitlines() if line.startswith("FAILED")]
-    verdict = "caught" if r.returncode else "SURVIVED"
-    return name, verdict + (" by " + failed[0].split()[1] if failed else "")
+    outcome = "caught" if r.returncode else "SURVIVED"
+    return name, outcome + (" by " + failed[0].split()[1] if failed else "")
 
 
 def main():

@@ -113,8 +113,8 @@ def run(name, tmp):
                         "-p", "no:cacheprovider"], cwd=d, env=env, capture_output=True,
                        text=True, timeout=900)
     failed = [line for line in r.stdout.splitlines() if line.startswith("FAILED")]
-    verdict = "caught" if r.returncode != 0 else "SURVIVED"
-    return name, verdict + (" by " + failed[0].split()[1] if failed else "")
+    outcome = "caught" if r.returncode != 0 else "SURVIVED"
+    return name, outcome + (" by " + failed[0].split()[1] if failed else "")
 
 
 def main():
