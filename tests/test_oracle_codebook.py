@@ -121,3 +121,8 @@ def test_bf16_rounding_matches_torch_cast():
     assert np.array_equal(ours, ref)
     nan_bits = O.bf16_bits_rne(np.array([np.nan], np.float32))
     assert np.isnan(O.bf16_bits_to_f32(nan_bits))[0]
+    # NaNs whose payload lies only in the 16 bits the rounding drops stay NaN (not infinity),
+    # as torch's cast keeps them NaN
+    odd = np.array([0x7F800001, 0xFF800001, 0x7F80FFFF, 0x7FFFFFFF], np.uint32).view(np.float32)
+    assert np.all(np.isnan(O.bf16_bits_to_f32(O.bf16_bits_rne(odd))))
+    assert torch.isnan(torch.from_numpy(odd).to(torch.bfloat16)).all()
